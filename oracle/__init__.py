@@ -1,0 +1,30 @@
+"""Plain fp64 CPU oracle for the FVAttn routing front end and block-sparse attention.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import this package:
+only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` use it. It shares no code with the
+CUDA library (``block_sparse_attention_video_b200``) and imports nothing from it.
+
+Sources (page title, section):
+  [FVAttn] "FVAttn: Adaptive Sparse Attention with Runtime Load Balancing for
+           Video Generation" (Liu et al.), read through its Chinese translation,
+           its English summary and its abstract page.
+  [GSRS]   "Sparse Attention for Video Generation Acceleration via Growing
+           Sparsity and Reduced Search".
+"""
+
+from .fvattn_oracle import (  # noqa: F401
+    num_blocks,
+    tile_order,
+    permute,
+    inverse_permute,
+    block_mean_pool,
+    block_scores,
+    topp_topk_select,
+    route,
+    selection_mask,
+    head_work,
+    masked_attention,
+    masked_attention_rows,
+    dense_attention,
+)
