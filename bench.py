@@ -1,0 +1,401 @@
+"""Benchmark of the block-sparse attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fvattn|reference]
+                    [--workload wan14b-720p] [--no-e2e] [--no-cpu-baseline]
+
+One step = one attention call of the whole path over one synthetic input
+already resident in HBM: route (tile permutation of Q and K fused with
+block-mean pooling, block scores, Top-p + Top-k floor, lists, per-head work),
+permutation of V, block-sparse attention, inverse permutation of the output.
+Throughput = effective TFLOP/s counted over the selected blocks only
+(4 * d * sum over selected (query block, key block) pairs of
+valid_query_rows * valid_keys), per step and per attention launch. The
+build's own dense kernel is timed beside it at the same shape.
+
+Multi-GPU (torchrun): every rank runs its own independent call (weak
+scaling, no collective on the data path); the timed region is bracketed by
+barriers and the max over ranks is reported.
+
+--impl reference times the fp64 oracle (the CPU reference of this method) on
+the host cores on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic as S  # noqa: E402
+
+METRIC = "sparse attn ms/call & effective TFLOP/s (Wan-14B 720p shape) vs own dense"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return dict(hbm=float(pk["hbm_gbs"]), bf16=float(pk["bf16_tflops"]),
+                    bf16_sus=float(pk["bf16_tflops_sustained"]), source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+def effective_flops(kv_idx: np.ndarray, kv_cnt: np.ndarray, N: int, bs: int, d: int) -> float:
+    """4*d*sum over selected (i, j) of valid_rows(i) * valid_keys(j)."""
+    nb = kv_cnt.shape[-1]
+    n = np.full(nb, bs, dtype=np.float64)
+    n[-1] = N - (nb - 1) * bs
+    valid = np.arange(kv_idx.shape[-1]) < kv_cnt[..., None]
+    keys = np.where(valid, n[np.clip(kv_idx, 0, nb - 1)], 0.0).sum(-1)      # [B,H,nb]
+    return float(4.0 * d * (keys * n[None, None, :]).sum())
+
+
+def dense_flops(B, H, N, d) -> float:
+    return 4.0 * B * H * float(N) * float(N) * d
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"fvattn_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9], float(parts[3])))
+                except ValueError:
+                    continue
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return None
+        load = [r for r in rows if r[3] > 200.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i, v in enumerate(r[2]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(load),
+                "power_w_max": max(r[3] for r in rows)}
+
+
+def _dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=120))
+        return dist, rank, world, local
+    torch.cuda.set_device(local)
+    return None, 0, 1, local
+
+
+def _barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def _max_over_ranks(dist, v: float) -> float:
+    if dist is None:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_oracle_sample(w, q, k, v, kv_idx, kv_cnt, budget_s=15.0, seed=0):
+    """Oracle masked attention on sampled query blocks of the GPU's mask; returns
+    (effective TFLOP/s, blocks, seconds, cores)."""
+    import oracle as O
+    cores = len(os.sched_getaffinity(0))
+    perm = O.tile_order(*w.grid6)
+    nb = w.nb
+    rng = np.random.default_rng(seed)
+    idx = kv_idx.cpu().numpy()
+    cnt = kv_cnt.cpu().numpy()
+    n = np.full(nb, w.block, dtype=np.float64)
+    n[-1] = w.N - (nb - 1) * w.block
+    scale = 1.0 / math.sqrt(w.d)
+    flops = 0.0
+    blocks = 0
+    t0 = time.perf_counter()
+    heads = rng.permutation(w.H)
+    for h in heads:
+        qh, kh, vh = (O.permute(x[0, h].float().cpu().numpy().astype(np.float64), perm, w.block)
+                      for x in (q, k, v))
+        for i in rng.permutation(nb)[:4]:
+            mrow = np.zeros(nb, dtype=bool)
+            mrow[idx[0, h, i, :cnt[0, h, i]]] = True
+            O.masked_attention_rows(qh, kh, vh, mrow, w.N, w.block, scale, int(i))
+            flops += 4.0 * w.d * n[i] * n[mrow].sum()
+            blocks += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return flops / dt / 1e12, blocks, dt, cores
+
+
+def run_fvattn(args):
+    import block_sparse_attention_video_b200 as F
+    dist, rank, world, local = _dist_setup(args.gpus)
+    w = S.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    q, k, v = S.make_qkv(w.replace(seed=w.seed + 1000 * rank), device=dev)
+    path = F.FVAttnPath(w.B, w.H, w.grid, w.tile, w.block, w.d, torch.bfloat16, w.p, w.k_min, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev_attn=None):
+        path.route(q, k)
+        F.fvattn_permute(v, path.vp, path.grid)
+        if ev_attn is not None:
+            ev_attn[0].record(stream)
+        path.attend()
+        if ev_attn is not None:
+            ev_attn[1].record(stream)
+        F.fvattn_permute(path.op, path.out, path.grid, inverse=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if F.fvattn_workspace_status(path.ws_route) != F.FVATTN_OK or \
+            F.fvattn_workspace_status(path.ws_attn) != F.FVATTN_OK:
+        raise RuntimeError("kernel status word set during warm-up")
+    idx_np, cnt_np = path.kv_idx.cpu().numpy(), path.kv_cnt.cpu().numpy()
+    eff = effective_flops(idx_np, cnt_np, w.N, w.block, w.d)
+    density = float(cnt_np.mean() / path.nb)
+    hw = path.head_work.cpu().numpy().astype(np.float64)
+    work_ratio = float(hw.max() / hw.mean())
+
+    # ---- timed region: K full steps, per-launch events around the attention kernel
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else local
+    with ClockSampler(gpu_index) as clk:
+        _barrier(dist)
+        torch.cuda.synchronize()
+        start.record(stream)
+        for s in range(args.steps):
+            step(ev[s])
+        end.record(stream)
+        torch.cuda.synchronize()
+        _barrier(dist)
+    clocks = clk.summary()
+    ms_step = start.elapsed_time(end) / args.steps
+    attn_ms = [a.elapsed_time(b) for a, b in ev]
+    ms_attn = sum(attn_ms) / len(attn_ms)
+    ms_step_max = _max_over_ranks(dist, ms_step)
+    launches_per_step = 7   # gather_pool, route_select, permute V, plan x2, attention, inverse permute
+
+    # ---- the build's own dense kernel at the same shape
+    dense_ms = []
+    for it in range(args.warmup + max(2, args.steps // 2)):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        path.attend(dense=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            dense_ms.append(a.elapsed_time(b))
+    ms_dense = sum(dense_ms) / len(dense_ms)
+    d_flops = dense_flops(w.B, w.H, w.N, w.d)
+
+    # ---- e2e through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+        hout = torch.empty(path.out.shape, dtype=path.out.dtype).pin_memory()
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            out = path(dq, dk, dv)
+            hout.copy_(out, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        e_steps = max(2, args.steps // 2)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        _barrier(dist)
+        a.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        _barrier(dist)
+        ms_e2e = _max_over_ranks(dist, a.elapsed_time(b) / e_steps)
+        in_bytes = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
+        e2e = {"value": world * eff / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms_e2e,
+               "h2d_bytes_per_step": int(in_bytes), "d2h_bytes_per_step": int(hout.numel() * hout.element_size())}
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return 0
+
+    pk = _peaks()
+    achieved = eff / (ms_attn * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": world * eff / (ms_step_max * 1e-3) / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "grid": list(w.grid),
+                   "tiles": list(w.tile), "block": w.block, "p": w.p, "k_min": w.k_min,
+                   "l2": "inputs larger than L2 (Q, K, V 774 MB each); no flush",
+                   "parallelism": f"independent replicas x{world}"},
+        "ms_per_call": ms_step_max,
+        "attention_ms_per_launch": ms_attn,
+        "effective_tflop_per_call": eff / 1e12,
+        "density": density,
+        "head_work_max_over_mean": work_ratio,
+        "dense": {"attention_ms_per_launch": ms_dense, "tflops": d_flops / (ms_dense * 1e-3) / 1e12,
+                  "tflop_per_call": d_flops / 1e12},
+        "speedup_vs_dense_attention": ms_dense / ms_attn,
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_sm100_kernel", "achieved": achieved,
+                     "peak": pk["bf16_sus"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_sus"],
+                     "peak_kind": f"{pk['source']} bf16 sustained (kernel timed inside a long step)",
+                     "frac_of_burst_peak": achieved / pk["bf16"], "traffic": None},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if not args.no_cpu_baseline:
+        tf, nblk, secs, cores = cpu_oracle_sample(w, q, k, v, path.kv_idx, path.kv_cnt,
+                                                  budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                "sample": f"fp64 oracle block-sparse attention of {nblk} query blocks "
+                                          f"(4 per head, random heads) of this call on the GPU's mask, "
+                                          f"{secs:.1f} s"}
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def run_reference(args):
+    """The oracle timed on the host cores on a bounded sample of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle as O
+    w = S.WORKLOADS[args.workload]
+    cores = len(os.sched_getaffinity(0))
+    q, k, v = S.make_qkv(w, device="cpu")
+    perm = O.tile_order(*w.grid6)
+    scale = 1.0 / math.sqrt(w.d)
+    nb = w.nb
+    n = np.full(nb, w.block, dtype=np.float64)
+    n[-1] = w.N - (nb - 1) * w.block
+    rng = np.random.default_rng(0)
+
+    def one_step(h):
+        # one head: route (permute, pool, scores, Top-p) + attention of 2 query blocks
+        qh, kh, vh = (O.permute(x[0, h].float().numpy().astype(np.float64), perm, w.block) for x in (q, k, v))
+        qbar, kbar = O.block_mean_pool(qh, w.N, w.block), O.block_mean_pool(kh, w.N, w.block)
+        s = O.block_scores(qbar, kbar, scale)
+        flops = 0.0
+        for i in rng.permutation(nb)[:2]:
+            order, c = O.topp_topk_select(s[i], w.p, w.k_min)
+            mrow = np.zeros(nb, dtype=bool)
+            mrow[order[:c]] = True
+            O.masked_attention_rows(qh, kh, vh, mrow, w.N, w.block, scale, int(i))
+            flops += 4.0 * w.d * n[i] * n[mrow].sum()
+        return flops
+
+    for h in range(args.warmup):
+        one_step(h % w.H)
+    t0 = time.perf_counter()
+    flops = 0.0
+    for s_ in range(args.steps):
+        flops += one_step((args.warmup + s_) % w.H)
+    dt = time.perf_counter() - t0
+    tf = flops / dt / 1e12
+    line = {"metric": METRIC, "value": tf, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "block": w.block,
+                       "p": w.p, "k_min": w.k_min},
+            "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": "per step: one head's fp64 routing (permute, pool, scores, "
+                                       "Top-p) and block-sparse attention of 2 query blocks"},
+            "e2e": {"value": tf, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("fvattn", "reference"), default="fvattn")
+    ap.add_argument("--workload", default="wan14b-720p", choices=sorted(S.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "fvattn":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    return run_reference(args) if args.impl == "reference" else run_fvattn(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,249 @@
+"""Python binding of libfvattn.so (include/fvattn.h): argument marshalling only.
+
+Every step of the attention path runs in the library's CUDA kernels; this
+module turns torch tensors into pointers and sizes, passes the current CUDA
+stream, and raises on a non-OK status. It never computes on the CPU and has no
+fallback: importing it fails loudly if the library has not been built
+(``python -m block_sparse_attention_video_b200.build_lib``).
+
+Entry points carry the C names: ``fvattn_permute``, ``fvattn_route``,
+``fvattn_sparse_fwd``, ``fvattn_dense_fwd``, ``fvattn_workspace_bytes``,
+``fvattn_workspace_status``. ``FVAttnPath`` strings them into the full per-call
+path (route -> permute V -> block-sparse attention -> inverse permute) over
+buffers it allocates once with torch.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfvattn.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with "
+        "`python -m block_sparse_attention_video_b200.build_lib` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+FVATTN_OK = 0
+FVATTN_ERR_INVALID_ARG = 1
+FVATTN_ERR_UNSUPPORTED = 2
+FVATTN_ERR_WORKSPACE = 3
+FVATTN_ERR_CUDA = 4
+FVATTN_ERR_TIMEOUT = 5
+
+FVATTN_BF16 = 0
+FVATTN_FP32 = 1
+
+FVATTN_OP_ROUTE = 0
+FVATTN_OP_SPARSE_FWD = 1
+FVATTN_OP_DENSE_FWD = 2
+
+EXPORTED = ("fvattn_workspace_bytes", "fvattn_permute", "fvattn_route", "fvattn_sparse_fwd",
+            "fvattn_dense_fwd", "fvattn_workspace_status", "fvattn_status_string")
+
+
+class Grid(ctypes.Structure):
+    """fvattn_grid: latent video grid (T, Hh, W), tiles (tt, th, tw), block size."""
+    _fields_ = [("T", ctypes.c_int), ("Hh", ctypes.c_int), ("W", ctypes.c_int),
+                ("tt", ctypes.c_int), ("th", ctypes.c_int), ("tw", ctypes.c_int),
+                ("block", ctypes.c_int)]
+
+    @classmethod
+    def make(cls, grid, tile, block):
+        return cls(*grid, *tile, block)
+
+    @property
+    def N(self):
+        return self.T * self.Hh * self.W
+
+    @property
+    def nb(self):
+        return -(-self.N // self.block)
+
+
+_c_int, _c_void_p, _c_float, _c_size_t = ctypes.c_int, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
+_lib.fvattn_workspace_bytes.argtypes = [_c_int] * 6
+_lib.fvattn_workspace_bytes.restype = _c_size_t
+_lib.fvattn_permute.argtypes = [_c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                ctypes.POINTER(Grid), _c_int, _c_void_p]
+_lib.fvattn_permute.restype = _c_int
+_lib.fvattn_route.argtypes = [_c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
+                              ctypes.POINTER(Grid), _c_float, _c_int, _c_void_p, _c_void_p,
+                              _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_void_p]
+_lib.fvattn_route.restype = _c_int
+_lib.fvattn_sparse_fwd.argtypes = [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                                   _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                   _c_int, _c_float, _c_void_p, _c_size_t, _c_void_p]
+_lib.fvattn_sparse_fwd.restype = _c_int
+_lib.fvattn_dense_fwd.argtypes = [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                                  _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
+                                  _c_void_p, _c_size_t, _c_void_p]
+_lib.fvattn_dense_fwd.restype = _c_int
+_lib.fvattn_workspace_status.argtypes = [_c_void_p, _c_void_p]
+_lib.fvattn_workspace_status.restype = _c_int
+_lib.fvattn_status_string.argtypes = [_c_int]
+_lib.fvattn_status_string.restype = ctypes.c_char_p
+
+
+class FVAttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {fvattn_status_string(status)} (status {status})")
+
+
+def fvattn_status_string(status: int) -> str:
+    return _lib.fvattn_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != FVATTN_OK:
+        raise FVAttnError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return FVATTN_BF16
+    if t.dtype == torch.float32:
+        return FVATTN_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def fvattn_workspace_bytes(op: int, B: int, H: int, N: int, d: int, block: int) -> int:
+    return int(_lib.fvattn_workspace_bytes(op, B, H, N, d, block))
+
+
+def fvattn_permute(x, y, grid: Grid, inverse: bool = False, stream=None):
+    """x [B,H,N,d] -> y [B,H,Npad,d] (tile order), or the inverse."""
+    _need_cuda(x, y)
+    B, H, _, d = x.shape
+    _check(_lib.fvattn_permute(_ptr(x), _ptr(y), B, H, grid.N, d, _dtype_code(x), ctypes.byref(grid),
+                               1 if inverse else 0, _stream(stream)), "fvattn_permute")
+    return y
+
+
+def fvattn_route(q, k, grid: Grid, p: float, k_min: int, kv_idx, kv_cnt, head_work, workspace,
+                 qp_out=None, kp_out=None, stream=None):
+    """Routing front end; fills kv_idx [B,H,nb,nb], kv_cnt [B,H,nb], head_work [B,H]."""
+    _need_cuda(q, k, kv_idx, kv_cnt, head_work, workspace, qp_out, kp_out)
+    B, H, N, d = q.shape
+    _check(_lib.fvattn_route(_ptr(q), _ptr(k), B, H, N, d, _dtype_code(q), ctypes.byref(grid),
+                             float(p), int(k_min), _ptr(qp_out), _ptr(kp_out), _ptr(kv_idx),
+                             _ptr(kv_cnt), _ptr(head_work), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream)),
+           "fvattn_route")
+    return kv_idx, kv_cnt, head_work
+
+
+def fvattn_sparse_fwd(qp, kp, vp, out, kv_idx, kv_cnt, N: int, block: int, workspace,
+                      scale=None, lse=None, stream=None):
+    """Block-sparse attention over permuted [B,H,Npad,d] tensors."""
+    _need_cuda(qp, kp, vp, out, kv_idx, kv_cnt, workspace, lse)
+    B, H, _, d = qp.shape
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(_lib.fvattn_sparse_fwd(_ptr(qp), _ptr(kp), _ptr(vp), _ptr(out), _ptr(lse), _ptr(kv_idx),
+                                  _ptr(kv_cnt), B, H, N, d, _dtype_code(qp), block, sc,
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  _stream(stream)), "fvattn_sparse_fwd")
+    return out
+
+
+def fvattn_dense_fwd(qp, kp, vp, out, N: int, block: int, workspace, scale=None, lse=None,
+                     stream=None):
+    """Dense attention over permuted [B,H,Npad,d] tensors (every key block)."""
+    _need_cuda(qp, kp, vp, out, workspace, lse)
+    B, H, _, d = qp.shape
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(_lib.fvattn_dense_fwd(_ptr(qp), _ptr(kp), _ptr(vp), _ptr(out), _ptr(lse), B, H, N, d,
+                                 _dtype_code(qp), block, sc, _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)),
+           "fvattn_dense_fwd")
+    return out
+
+
+def fvattn_workspace_status(workspace, stream=None) -> int:
+    """Synchronize the stream and return the status word the kernels recorded."""
+    return int(_lib.fvattn_workspace_status(_ptr(workspace), _stream(stream)))
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    """A 256-byte aligned uint8 buffer (torch's caching allocator aligns to 512)."""
+    t = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    assert t.data_ptr() % 256 == 0
+    return t
+
+
+class FVAttnPath:
+    """The whole per-call path on one device with buffers allocated once.
+
+    ``__call__(q, k, v)`` takes [B,H,N,d] tensors in original token order and
+    returns the attention output [B,H,N,d] in original order: route (which
+    also permutes q and k), permute v, block-sparse attention, inverse permute.
+    ``dense=True`` runs the dense kernel instead of routing.
+    """
+
+    def __init__(self, B, H, grid, tile, block, d, dtype, p, k_min, device="cuda"):
+        self.grid = Grid.make(grid, tile, block)
+        self.B, self.H, self.d = B, H, d
+        self.N, self.nb = self.grid.N, self.grid.nb
+        self.npad = self.nb * block
+        self.block = block
+        self.p, self.k_min = float(p), int(k_min)
+        self.dtype = dtype
+        dev = torch.device(device)
+        shp = (B, H, self.npad, d)
+        self.qp = torch.empty(shp, dtype=dtype, device=dev)
+        self.kp = torch.empty(shp, dtype=dtype, device=dev)
+        self.vp = torch.empty(shp, dtype=dtype, device=dev)
+        self.op = torch.empty(shp, dtype=dtype, device=dev)
+        self.out = torch.empty((B, H, self.N, d), dtype=dtype, device=dev)
+        self.kv_idx = torch.empty((B, H, self.nb, self.nb), dtype=torch.int32, device=dev)
+        self.kv_cnt = torch.empty((B, H, self.nb), dtype=torch.int32, device=dev)
+        self.head_work = torch.empty((B, H), dtype=torch.int64, device=dev)
+        self.ws_route = alloc_workspace(
+            fvattn_workspace_bytes(FVATTN_OP_ROUTE, B, H, self.N, d, block), dev)
+        self.ws_attn = alloc_workspace(
+            fvattn_workspace_bytes(FVATTN_OP_SPARSE_FWD, B, H, self.N, d, block), dev)
+
+    def route(self, q, k):
+        fvattn_route(q, k, self.grid, self.p, self.k_min, self.kv_idx, self.kv_cnt,
+                     self.head_work, self.ws_route, qp_out=self.qp, kp_out=self.kp)
+
+    def attend(self, dense=False):
+        if dense:
+            fvattn_dense_fwd(self.qp, self.kp, self.vp, self.op, self.N, self.block, self.ws_attn)
+        else:
+            fvattn_sparse_fwd(self.qp, self.kp, self.vp, self.op, self.kv_idx, self.kv_cnt,
+                              self.N, self.block, self.ws_attn)
+
+    def __call__(self, q, k, v, dense=False):
+        if dense:
+            fvattn_permute(q, self.qp, self.grid)
+            fvattn_permute(k, self.kp, self.grid)
+        else:
+            self.route(q, k)
+        fvattn_permute(v, self.vp, self.grid)
+        self.attend(dense=dense)
+        fvattn_permute(self.op, self.out, self.grid, inverse=True)
+        return self.out

@@ -1,0 +1,302 @@
+// api.cu -- the extern "C" entry points of libfvattn.so (declared in
+// include/fvattn.h): host-side validation, workspace layout, TMA tensor maps
+// and kernel dispatch. No entry point allocates device memory.
+#include <cmath>
+#include <cstdint>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+
+namespace fvattn {
+cudaError_t launch_permute(const void* x, void* y, int BH, int N, int d, int esize, int bs,
+                           const TileGeom& g, int inverse, cudaStream_t st);
+cudaError_t launch_gather_pool(const void* q, const void* k, void* qp, void* kp, float* qbar,
+                               float* kbar, int BH, int N, int d, bool bf16, int bs,
+                               const TileGeom& g, cudaStream_t st);
+int route_select_rows_per_warp(int nb, int d);
+cudaError_t launch_route_select(const float* qbar, const float* kbar, int BH, int nb, int d,
+                                float scale, float p, int k_min, int* kv_idx, int* kv_cnt,
+                                unsigned long long* head_work, int* status, cudaStream_t st);
+cudaError_t launch_attn_simt(const void* q, const void* k, const void* v, void* o, float* lse,
+                             const int* kv_idx, const int* kv_cnt, int BH, int N, int d, int bs,
+                             bool bf16, float scale, int* status, cudaStream_t st);
+cudaError_t launch_attn_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                              void* out, float* lse, const int* kv_idx, const int* kv_cnt,
+                              int* local_order, unsigned long long* head_total, int* head_order,
+                              int BH, int N, int nb, float scale, int* status,
+                              unsigned long long* counter, int num_sms, cudaStream_t st);
+}  // namespace fvattn
+
+namespace {
+
+using fvattn::align_up;
+using fvattn::kWsHeaderBytes;
+
+constexpr int kMaxBlocks = 4096;   // nb limit (route rows live in shared memory)
+constexpr int kMaxHeads = 4096;    // B*H limit (the work planner sorts heads in shared memory)
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+bool valid_dtype(fvattn_dtype dt) { return dt == FVATTN_BF16 || dt == FVATTN_FP32; }
+int elem_size(fvattn_dtype dt) { return dt == FVATTN_BF16 ? 2 : 4; }
+bool valid_d(int d) { return d == 64 || d == 128; }
+bool valid_block(int b) { return b == 64 || b == 128; }
+
+bool valid_sizes(int B, int H, int N, int d, int block) {
+  if (B < 1 || H < 1 || N < 1 || !valid_d(d) || !valid_block(block)) return false;
+  const long long bh = static_cast<long long>(B) * H;
+  if (bh > kMaxHeads) return false;
+  const long long nb = (static_cast<long long>(N) + block - 1) / block;
+  if (nb > kMaxBlocks) return false;
+  return true;
+}
+
+int num_blocks(int N, int block) { return (N + block - 1) / block; }
+
+// ------------------------------------------------------------- workspace layout
+struct RouteWs {
+  size_t qbar, kbar, total;
+};
+RouteWs route_ws(int B, int H, int N, int d, int block) {
+  const size_t bars = static_cast<size_t>(B) * H * num_blocks(N, block) * d * sizeof(float);
+  RouteWs w;
+  w.qbar = kWsHeaderBytes;
+  w.kbar = w.qbar + align_up(bars, 256);
+  w.total = w.kbar + align_up(bars, 256);
+  return w;
+}
+
+struct AttnWs {
+  size_t local_order, head_total, head_order, total;
+};
+AttnWs sparse_ws(int B, int H, int N, int block) {
+  const size_t bh = static_cast<size_t>(B) * H;
+  AttnWs w;
+  w.local_order = kWsHeaderBytes;
+  w.head_total = w.local_order + align_up(bh * num_blocks(N, block) * sizeof(int), 256);
+  w.head_order = w.head_total + align_up(bh * sizeof(unsigned long long), 256);
+  w.total = w.head_order + align_up(bh * sizeof(int), 256);
+  return w;
+}
+
+// ------------------------------------------------------------- device properties
+int device_sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// [rows, 128] bf16, row stride 256 B; box = 128 rows x 64 columns, 128-byte swizzle.
+bool make_row_map(CUtensorMap* map, const void* base, uint64_t rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {256};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+fvattn_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA; }
+
+fvattn::TileGeom geom_of(const fvattn_grid* g) {
+  return fvattn::TileGeom{g->T, g->Hh, g->W, g->tt, g->th, g->tw};
+}
+
+bool valid_grid(const fvattn_grid* g, int N) {
+  if (!g) return false;
+  if (g->T < 1 || g->Hh < 1 || g->W < 1 || g->tt < 1 || g->th < 1 || g->tw < 1) return false;
+  if (!valid_block(g->block)) return false;
+  const long long n = static_cast<long long>(g->T) * g->Hh * g->W;
+  return n == N;
+}
+
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+fvattn_status check_ws(const void* ws, size_t have, size_t need) {
+  if (!ws || !aligned(ws, 256) || have < need) return FVATTN_ERR_WORKSPACE;
+  return FVATTN_OK;
+}
+
+// Common validation and dispatch of the attention forward (sparse or dense).
+fvattn_status attention_fwd(const void* qp, const void* kp, const void* vp, void* op, float* lse,
+                            const int32_t* kv_idx, const int32_t* kv_cnt, bool sparse, int B,
+                            int H, int N, int d, fvattn_dtype dtype, int block, float scale,
+                            void* ws, size_t ws_bytes, void* stream) {
+  if (!qp || !kp || !vp || !op) return FVATTN_ERR_INVALID_ARG;
+  if (!aligned(qp, 16) || !aligned(kp, 16) || !aligned(vp, 16) || !aligned(op, 16))
+    return FVATTN_ERR_INVALID_ARG;
+  if (lse && !aligned(lse, 4)) return FVATTN_ERR_INVALID_ARG;
+  if (sparse && (!kv_idx || !kv_cnt || !aligned(kv_idx, 4) || !aligned(kv_cnt, 4)))
+    return FVATTN_ERR_INVALID_ARG;
+  if (!valid_dtype(dtype) || !valid_sizes(B, H, N, d, block)) return FVATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FVATTN_ERR_INVALID_ARG;
+  const size_t need = fvattn_workspace_bytes(sparse ? FVATTN_OP_SPARSE_FWD : FVATTN_OP_DENSE_FWD,
+                                             B, H, N, d, block);
+  const fvattn_status wst = check_ws(ws, ws_bytes, need);
+  if (wst != FVATTN_OK) return wst;
+
+  auto st = static_cast<cudaStream_t>(stream);
+  auto base = static_cast<uint8_t*>(ws);
+  auto hdr = reinterpret_cast<fvattn::WsHeader*>(base);
+  const int BH = B * H;
+  const int nb = num_blocks(N, block);
+  if (cudaMemsetAsync(base, 0, kWsHeaderBytes, st) != cudaSuccess) return FVATTN_ERR_CUDA;
+
+  const bool tensor_core = dtype == FVATTN_BF16 && d == 128 && block == 128;
+  if (!tensor_core) {
+    return from_cuda(fvattn::launch_attn_simt(qp, kp, vp, op, lse, sparse ? kv_idx : nullptr,
+                                              sparse ? kv_cnt : nullptr, BH, N, d, block,
+                                              dtype == FVATTN_BF16, scale, &hdr->status, st));
+  }
+  const uint64_t rows = static_cast<uint64_t>(BH) * nb * block;
+  CUtensorMap tq, tk, tv;
+  if (!make_row_map(&tq, qp, rows) || !make_row_map(&tk, kp, rows) || !make_row_map(&tv, vp, rows))
+    return FVATTN_ERR_CUDA;
+  const int sms = device_sm_count();
+  if (sms <= 0) return FVATTN_ERR_CUDA;
+  int* local_order = nullptr;
+  unsigned long long* head_total = nullptr;
+  int* head_order = nullptr;
+  if (sparse) {
+    const AttnWs w = sparse_ws(B, H, N, block);
+    local_order = reinterpret_cast<int*>(base + w.local_order);
+    head_total = reinterpret_cast<unsigned long long*>(base + w.head_total);
+    head_order = reinterpret_cast<int*>(base + w.head_order);
+  }
+  return from_cuda(fvattn::launch_attn_sm100(
+      tq, tk, tv, op, lse, sparse ? kv_idx : nullptr, sparse ? kv_cnt : nullptr, local_order,
+      head_total, head_order, BH, N, nb, scale, &hdr->status, &hdr->counter, sms, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fvattn_workspace_bytes(fvattn_op op, int B, int H, int N, int d, int block) {
+  if (!valid_sizes(B, H, N, d, block)) return 0;
+  switch (op) {
+    case FVATTN_OP_ROUTE: return route_ws(B, H, N, d, block).total;
+    case FVATTN_OP_SPARSE_FWD: return sparse_ws(B, H, N, block).total;
+    case FVATTN_OP_DENSE_FWD: return kWsHeaderBytes;
+  }
+  return 0;
+}
+
+fvattn_status fvattn_permute(const void* x, void* y, int B, int H, int N, int d,
+                             fvattn_dtype dtype, const fvattn_grid* grid, int inverse,
+                             void* stream) {
+  if (!x || !y || !aligned(x, 16) || !aligned(y, 16)) return FVATTN_ERR_INVALID_ARG;
+  if (!valid_dtype(dtype) || !valid_grid(grid, N)) return FVATTN_ERR_INVALID_ARG;
+  if (!valid_sizes(B, H, N, d, grid->block)) return FVATTN_ERR_INVALID_ARG;
+  const int es = elem_size(dtype);
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t orig_bytes = bh * N * d * es;
+  const size_t perm_bytes = bh * num_blocks(N, grid->block) * grid->block * d * es;
+  if (ranges_overlap(x, inverse ? perm_bytes : orig_bytes, y, inverse ? orig_bytes : perm_bytes))
+    return FVATTN_ERR_INVALID_ARG;
+  return from_cuda(fvattn::launch_permute(x, y, B * H, N, d, es, grid->block, geom_of(grid),
+                                          inverse ? 1 : 0, static_cast<cudaStream_t>(stream)));
+}
+
+fvattn_status fvattn_route(const void* q, const void* k, int B, int H, int N, int d,
+                           fvattn_dtype dtype, const fvattn_grid* grid, float p, int k_min,
+                           void* qp_out, void* kp_out, int32_t* kv_idx, int32_t* kv_cnt,
+                           int64_t* head_work, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  if (!q || !k || !kv_idx || !kv_cnt || !head_work) return FVATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(kv_idx, 4) || !aligned(kv_cnt, 4) ||
+      !aligned(head_work, 8))
+    return FVATTN_ERR_INVALID_ARG;
+  if ((qp_out && !aligned(qp_out, 16)) || (kp_out && !aligned(kp_out, 16)))
+    return FVATTN_ERR_INVALID_ARG;
+  if (!valid_dtype(dtype) || !valid_grid(grid, N)) return FVATTN_ERR_INVALID_ARG;
+  if (!valid_sizes(B, H, N, d, grid->block)) return FVATTN_ERR_INVALID_ARG;
+  if (!(p > 0.f && p <= 1.f) || k_min < 1) return FVATTN_ERR_INVALID_ARG;
+  const int block = grid->block;
+  const int nb = num_blocks(N, block);
+  if (fvattn::route_select_rows_per_warp(nb, d) == 0) return FVATTN_ERR_UNSUPPORTED;
+  const RouteWs w = route_ws(B, H, N, d, block);
+  const fvattn_status wst = check_ws(workspace, workspace_bytes, w.total);
+  if (wst != FVATTN_OK) return wst;
+
+  auto st = static_cast<cudaStream_t>(stream);
+  auto base = static_cast<uint8_t*>(workspace);
+  auto hdr = reinterpret_cast<fvattn::WsHeader*>(base);
+  float* qbar = reinterpret_cast<float*>(base + w.qbar);
+  float* kbar = reinterpret_cast<float*>(base + w.kbar);
+  const int BH = B * H;
+  if (cudaMemsetAsync(base, 0, kWsHeaderBytes, st) != cudaSuccess) return FVATTN_ERR_CUDA;
+  if (cudaMemsetAsync(head_work, 0, sizeof(int64_t) * BH, st) != cudaSuccess)
+    return FVATTN_ERR_CUDA;
+  cudaError_t e = fvattn::launch_gather_pool(q, k, qp_out, kp_out, qbar, kbar, BH, N, d,
+                                             dtype == FVATTN_BF16, block, geom_of(grid), st);
+  if (e != cudaSuccess) return FVATTN_ERR_CUDA;
+  const float scale = 1.0f / std::sqrt(static_cast<float>(d));
+  e = fvattn::launch_route_select(qbar, kbar, BH, nb, d, scale, p, k_min, kv_idx, kv_cnt,
+                                  reinterpret_cast<unsigned long long*>(head_work), &hdr->status,
+                                  st);
+  return from_cuda(e);
+}
+
+fvattn_status fvattn_sparse_fwd(const void* qp, const void* kp, const void* vp, void* op,
+                                float* lse, const int32_t* kv_idx, const int32_t* kv_cnt, int B,
+                                int H, int N, int d, fvattn_dtype dtype, int block, float scale,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  return attention_fwd(qp, kp, vp, op, lse, kv_idx, kv_cnt, true, B, H, N, d, dtype, block,
+                       scale, workspace, workspace_bytes, stream);
+}
+
+fvattn_status fvattn_dense_fwd(const void* qp, const void* kp, const void* vp, void* op,
+                               float* lse, int B, int H, int N, int d, fvattn_dtype dtype,
+                               int block, float scale, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  return attention_fwd(qp, kp, vp, op, lse, nullptr, nullptr, false, B, H, N, d, dtype, block,
+                       scale, workspace, workspace_bytes, stream);
+}
+
+fvattn_status fvattn_workspace_status(const void* workspace, void* stream) {
+  if (!workspace || !aligned(workspace, 256)) return FVATTN_ERR_WORKSPACE;
+  int h = 0;
+  auto st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&h, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return FVATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FVATTN_ERR_CUDA;
+  return static_cast<fvattn_status>(h);
+}
+
+const char* fvattn_status_string(fvattn_status s) {
+  switch (s) {
+    case FVATTN_OK: return "ok";
+    case FVATTN_ERR_INVALID_ARG: return "invalid argument";
+    case FVATTN_ERR_UNSUPPORTED: return "unsupported shape";
+    case FVATTN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case FVATTN_ERR_CUDA: return "CUDA runtime error";
+    case FVATTN_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,168 @@
+/*
+ * fvattn.h -- C ABI of libfvattn.so: the data-parallel hot path of training-free
+ * adaptive block-sparse self-attention for video DiTs, built for NVIDIA B200
+ * (sm_100a).
+ *
+ * Sources (page title, section):
+ *   [FVAttn] "FVAttn: Adaptive Sparse Attention with Runtime Load Balancing for
+ *            Video Generation" (Liu et al.; Chinese translation, English summary
+ *            and abstract pages).
+ *   [GSRS]   "Sparse Attention for Video Generation Acceleration via Growing
+ *            Sparsity and Reduced Search".
+ *
+ * The path, per attention call of one layer:
+ *   fvattn_route      3-D tile permutation of Q and K, block-mean pooling, block
+ *                     score softmax, Top-p selection with a Top-k floor, KV block
+ *                     lists and per-head work            [FVAttn §2.1, §2.2, §3.1]
+ *   fvattn_permute    the same permutation for V (forward) and, inverse, for the
+ *                     attention output                   [FVAttn §3.1]
+ *   fvattn_sparse_fwd block-sparse attention over the routed lists
+ *                                                        [FVAttn §2.1; GSRS §3.2, §A.1]
+ *   fvattn_dense_fwd  the same kernel with every block selected (the dense
+ *                     baseline every page compares against)
+ *
+ * Conventions (every entry point):
+ *   - Tensors are dense, row-major, on the current CUDA device. A token row of
+ *     d elements is contiguous. Shapes are given in the comments as [B,H,N,d].
+ *   - N = T*Hh*W tokens in raster (t, y, x) order. nb = ceil(N/block) blocks;
+ *     Npad = nb*block. "Permuted" tensors are [B,H,Npad,d] in tile order with
+ *     the last Npad-N rows zero (written by fvattn_route / fvattn_permute).
+ *   - The caller owns every buffer, including the workspace; the library never
+ *     allocates or frees device memory and keeps no global state beyond a
+ *     per-device cache of device properties.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and never synchronizes the host, except
+ *     fvattn_workspace_status.
+ *   - Arguments are validated on the host before any launch: null pointers,
+ *     16-byte alignment of tensor pointers, shapes, dtype, block size, p and
+ *     k_min. On failure nothing is launched and a status is returned.
+ *   - Kernels never trap. A kernel that meets an out-of-range list entry clamps
+ *     it and records FVATTN_ERR_INVALID_ARG in the workspace status word; a
+ *     bounded wait that runs out records FVATTN_ERR_TIMEOUT there and the kernel
+ *     returns. fvattn_workspace_status reads that word back.
+ *   - No exception crosses this ABI.
+ */
+#ifndef FVATTN_H_
+#define FVATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FVATTN_API __attribute__((visibility("default")))
+#else
+#define FVATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FVATTN_OK = 0,
+  FVATTN_ERR_INVALID_ARG = 1, /* bad pointer, shape or parameter            */
+  FVATTN_ERR_UNSUPPORTED = 2, /* valid but not implemented for this shape    */
+  FVATTN_ERR_WORKSPACE = 3,   /* workspace missing, misaligned or too small  */
+  FVATTN_ERR_CUDA = 4,        /* a CUDA runtime call failed                  */
+  FVATTN_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out          */
+} fvattn_status;
+
+typedef enum {
+  FVATTN_BF16 = 0, /* tensor-core path (d = 128, block = 128) and SIMT path */
+  FVATTN_FP32 = 1  /* SIMT path only (fp32 arithmetic throughout)           */
+} fvattn_dtype;
+
+/* Latent video grid and tiling [FVAttn §3.1, read as 3-D tiles]. */
+typedef struct {
+  int T, Hh, W;   /* grid extents; N = T*Hh*W                               */
+  int tt, th, tw; /* tile extents (>= 1); edge tiles may be partial          */
+  int block;      /* tokens per block: 64 or 128                            */
+} fvattn_grid;
+
+typedef enum {
+  FVATTN_OP_ROUTE = 0,
+  FVATTN_OP_SPARSE_FWD = 1,
+  FVATTN_OP_DENSE_FWD = 2
+} fvattn_op;
+
+/* Workspace bytes needed by `op` for these sizes (0 if the sizes are invalid).
+ * The workspace must be 256-byte aligned. Its first 256 bytes hold the status
+ * word, cleared at the start of every call that takes it. */
+FVATTN_API size_t fvattn_workspace_bytes(fvattn_op op, int B, int H, int N, int d, int block);
+
+/* 3-D tile permutation [FVAttn §3.1].
+ * inverse == 0: x [B,H,N,d] (original order) -> y [B,H,Npad,d] (tile order,
+ *               pad rows zeroed).
+ * inverse != 0: x [B,H,Npad,d] (tile order)  -> y [B,H,N,d] (original order,
+ *               pad rows dropped).
+ * Token at grid (t,y,x) moves to position pos(t,y,x): tiles in raster order
+ * over the tile grid, raster order inside a tile. x and y must not overlap.
+ * d in {64, 128}; dtype BF16 or FP32. Bit-exact copy. */
+FVATTN_API fvattn_status fvattn_permute(const void* x, void* y, int B, int H, int N, int d,
+                             fvattn_dtype dtype, const fvattn_grid* grid,
+                             int inverse, void* stream);
+
+/* Routing front end [FVAttn §2.1, §2.2 Eq. (1), §3.1; GSRS §5.2, §5.3, §A.4].
+ * q, k      [B,H,N,d] in ORIGINAL token order.
+ * qp_out, kp_out  optional (NULL to skip) [B,H,Npad,d]: q and k permuted to
+ *           tile order, written by the same pass that pools them.
+ * Per (b,h) and query block i (blocks of the permuted sequence):
+ *   qbar_i, kbar_j = fp32 means over the valid tokens of each block;
+ *   s_ij = softmax_j(qbar_i . kbar_j / sqrt(d))  (fp32, max-subtracted);
+ *   n_p  = the smallest c such that the c largest s_ij sum to >= p
+ *          (nb when p >= 1 or when no prefix reaches p);
+ *   cnt  = min(nb, max(n_p, k_min)); the selected blocks are the cnt largest
+ *          (ties: lower block index ranks first).
+ * Outputs:
+ *   kv_idx    [B,H,nb,nb] int32: row (b,h,i) holds its cnt selected key blocks
+ *             in ascending block index at entries [0, cnt); entries >= cnt are
+ *             not written.
+ *   kv_cnt    [B,H,nb] int32: cnt per query block.
+ *   head_work [B,H] int64: sum_i cnt = nb * L_h of Eq. (1).
+ * 0 < p <= 1, k_min >= 1, d in {64,128}, block in {64,128}, N = T*Hh*W,
+ * nb <= 4096. Workspace: fvattn_workspace_bytes(FVATTN_OP_ROUTE, ...). */
+FVATTN_API fvattn_status fvattn_route(const void* q, const void* k, int B, int H, int N, int d,
+                           fvattn_dtype dtype, const fvattn_grid* grid, float p,
+                           int k_min, void* qp_out, void* kp_out, int32_t* kv_idx,
+                           int32_t* kv_cnt, int64_t* head_work, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* Block-sparse attention forward [FVAttn §2.1; GSRS §3.2, §A.1].
+ * qp, kp, vp [B,H,Npad,d] in tile order (pad rows zero), op [B,H,Npad,d] out.
+ * For every query token of query block i: softmax over the valid keys (index
+ * < N) of the key blocks kv_idx[b,h,i,0..cnt) of scale * q.k, times V.
+ * lse: optional [B,H,Npad] fp32 natural-log sum of exp of the scaled logits
+ * over the attended keys (NULL to skip). Rows >= N of op and lse are written
+ * but carry no meaning. kv_idx/kv_cnt as produced by fvattn_route (any order
+ * of entries within a row is accepted). scale > 0 (1/sqrt(d) is the usual).
+ * BF16 with d == 128 and block == 128 runs the tcgen05/TMEM tensor-core kernel
+ * (bf16 MMA, fp32 accumulation and softmax, P rounded to bf16); other shapes
+ * and FP32 run the SIMT kernel (fp32 throughout).
+ * Workspace: fvattn_workspace_bytes(FVATTN_OP_SPARSE_FWD, ...). */
+FVATTN_API fvattn_status fvattn_sparse_fwd(const void* qp, const void* kp, const void* vp,
+                                void* op, float* lse, const int32_t* kv_idx,
+                                const int32_t* kv_cnt, int B, int H, int N, int d,
+                                fvattn_dtype dtype, int block, float scale,
+                                void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/* Dense attention forward: fvattn_sparse_fwd with every key block selected.
+ * Workspace: fvattn_workspace_bytes(FVATTN_OP_DENSE_FWD, ...). */
+FVATTN_API fvattn_status fvattn_dense_fwd(const void* qp, const void* kp, const void* vp,
+                               void* op, float* lse, int B, int H, int N, int d,
+                               fvattn_dtype dtype, int block, float scale,
+                               void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* Synchronizes `stream` and returns the status word that the kernels of the
+ * last call using `workspace` recorded (FVATTN_OK if none). */
+FVATTN_API fvattn_status fvattn_workspace_status(const void* workspace, void* stream);
+
+/* Static string for a status code (never NULL). */
+FVATTN_API const char* fvattn_status_string(fvattn_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FVATTN_H_ */

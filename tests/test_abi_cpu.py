@@ -1,0 +1,135 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments with a status before any launch."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_video_b200 as F
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"FVATTN_API\s+[\w\s\*]+?\b(fvattn_\w+)\s*\(", src))
+    return sorted(names)
+
+
+def test_header_declares_the_four_calls_and_helpers():
+    decl = _declared_symbols()
+    for name in ("fvattn_permute", "fvattn_route", "fvattn_sparse_fwd", "fvattn_dense_fwd",
+                 "fvattn_workspace_bytes", "fvattn_workspace_status", "fvattn_status_string"):
+        assert name in decl
+
+
+@pytest.mark.parametrize("name", _declared_symbols())
+def test_library_exports_every_declared_symbol(name):
+    lib = ctypes.CDLL(F.LIB_PATH)
+    assert hasattr(lib, name)
+
+
+def test_status_strings():
+    for code in range(6):
+        assert F.fvattn_status_string(code)
+    assert F.fvattn_status_string(99) == "unknown status"
+
+
+def test_workspace_bytes():
+    assert F.fvattn_workspace_bytes(F.FVATTN_OP_DENSE_FWD, 1, 40, 75600, 128, 128) == 256
+    nb = 591
+    route = F.fvattn_workspace_bytes(F.FVATTN_OP_ROUTE, 1, 40, 75600, 128, 128)
+    assert route >= 256 + 2 * 40 * nb * 128 * 4
+    sparse = F.fvattn_workspace_bytes(F.FVATTN_OP_SPARSE_FWD, 1, 40, 75600, 128, 128)
+    assert sparse >= 256 + 40 * nb * 4 + 40 * 12
+    assert F.fvattn_workspace_bytes(F.FVATTN_OP_ROUTE, 1, 40, 75600, 96, 128) == 0   # bad d
+    assert F.fvattn_workspace_bytes(F.FVATTN_OP_ROUTE, 1, 40, 75600, 128, 32) == 0   # bad block
+    assert F.fvattn_workspace_bytes(F.FVATTN_OP_ROUTE, 0, 40, 75600, 128, 128) == 0
+
+
+FAKE = 1 << 20          # 16-byte aligned non-null address; never dereferenced (validation fails first)
+
+
+def _grid(**kw):
+    g = dict(T=4, Hh=8, W=8, tt=1, th=8, tw=8, block=64)
+    g.update(kw)
+    return F.Grid(g["T"], g["Hh"], g["W"], g["tt"], g["th"], g["tw"], g["block"])
+
+
+def _permute(x=FAKE, y=FAKE * 4, N=256, d=64, dt=F.FVATTN_FP32, grid=None):
+    g = grid if grid is not None else _grid()
+    return F._lib.fvattn_permute(x, y, 1, 2, N, d, dt, ctypes.byref(g), 0, None)
+
+
+@pytest.mark.parametrize("kw, status", [
+    (dict(x=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(y=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(x=FAKE + 4), F.FVATTN_ERR_INVALID_ARG),          # misaligned
+    (dict(N=255), F.FVATTN_ERR_INVALID_ARG),               # N != T*Hh*W
+    (dict(d=96), F.FVATTN_ERR_INVALID_ARG),
+    (dict(dt=7), F.FVATTN_ERR_INVALID_ARG),
+    (dict(grid=_grid(tt=0)), F.FVATTN_ERR_INVALID_ARG),
+    (dict(grid=_grid(block=32)), F.FVATTN_ERR_INVALID_ARG),
+    (dict(y=FAKE + 1024), F.FVATTN_ERR_INVALID_ARG),       # overlapping buffers
+])
+def test_permute_rejects(kw, status):
+    assert _permute(**kw) == status
+
+
+def _route(q=FAKE, k=FAKE, p=0.9, k_min=1, ws=FAKE, ws_bytes=1 << 30, idx=FAKE, cnt=FAKE,
+           hw=FAKE, grid=None, N=256, d=64):
+    g = grid if grid is not None else _grid()
+    return F._lib.fvattn_route(q, k, 1, 2, N, d, F.FVATTN_FP32, ctypes.byref(g), p, k_min, None,
+                               None, idx, cnt, hw, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw, status", [
+    (dict(q=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(idx=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(hw=FAKE + 4), F.FVATTN_ERR_INVALID_ARG),
+    (dict(p=0.0), F.FVATTN_ERR_INVALID_ARG),
+    (dict(p=1.5), F.FVATTN_ERR_INVALID_ARG),
+    (dict(p=float("nan")), F.FVATTN_ERR_INVALID_ARG),
+    (dict(k_min=0), F.FVATTN_ERR_INVALID_ARG),
+    (dict(ws=None), F.FVATTN_ERR_WORKSPACE),
+    (dict(ws=FAKE + 16), F.FVATTN_ERR_WORKSPACE),
+    (dict(ws_bytes=100), F.FVATTN_ERR_WORKSPACE),
+    (dict(grid=_grid(T=4096, Hh=128, W=1, th=8, tw=1), N=4096 * 128), F.FVATTN_ERR_INVALID_ARG),
+])
+def test_route_rejects(kw, status):
+    assert _route(**kw) == status
+
+
+def _sparse(qp=FAKE, op=FAKE, idx=FAKE, scale=0.125, ws=FAKE, ws_bytes=1 << 30, B=1, H=2, N=256,
+            d=64, block=64, dt=F.FVATTN_FP32):
+    return F._lib.fvattn_sparse_fwd(qp, FAKE, FAKE, op, None, idx, FAKE, B, H, N, d, dt, block,
+                                    scale, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw, status", [
+    (dict(qp=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(idx=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(op=FAKE + 8), F.FVATTN_ERR_INVALID_ARG),
+    (dict(scale=0.0), F.FVATTN_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), F.FVATTN_ERR_INVALID_ARG),
+    (dict(d=32), F.FVATTN_ERR_INVALID_ARG),
+    (dict(block=256), F.FVATTN_ERR_INVALID_ARG),
+    (dict(B=0), F.FVATTN_ERR_INVALID_ARG),
+    (dict(B=100, H=100), F.FVATTN_ERR_INVALID_ARG),        # B*H above the planner's limit
+    (dict(ws_bytes=16), F.FVATTN_ERR_WORKSPACE),
+    (dict(ws=None), F.FVATTN_ERR_WORKSPACE),
+])
+def test_sparse_rejects(kw, status):
+    assert _sparse(**kw) == status
+
+
+def test_dense_rejects_and_status_rejects_bad_workspace():
+    assert F._lib.fvattn_dense_fwd(FAKE, FAKE, FAKE, None, None, 1, 1, 256, 64, F.FVATTN_FP32, 64,
+                                   0.125, FAKE, 1 << 20, None) == F.FVATTN_ERR_INVALID_ARG
+    assert F._lib.fvattn_workspace_status(None, None) == F.FVATTN_ERR_WORKSPACE
+    assert F._lib.fvattn_workspace_status(FAKE + 64, None) == F.FVATTN_ERR_WORKSPACE
