@@ -22,8 +22,9 @@ cudaError_t launch_attn_simt(const void* q, const void* k, const void* v, void* 
                              bool bf16, float scale, int* status, cudaStream_t st);
 cudaError_t launch_attn_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                               void* out, float* lse, const int* kv_idx, const int* kv_cnt,
-                              int* local_order, unsigned long long* head_total, int* head_order,
-                              int BH, int N, int nb, float scale, int* status,
+                              uint32_t* ulist, int* ucnt, int* local_order,
+                              unsigned long long* head_total, int* head_order, int BH, int N,
+                              int nb, int bs, float scale, int* status,
                               unsigned long long* counter, int num_sms, cudaStream_t st);
 }  // namespace fvattn
 
@@ -65,14 +66,20 @@ RouteWs route_ws(int B, int H, int N, int d, int block) {
   return w;
 }
 
+// The tensor-core kernel works on units of 256 query rows = 256/block query
+// blocks; the sparse path first merges each unit's KV lists into one union list.
 struct AttnWs {
-  size_t local_order, head_total, head_order, total;
+  size_t ulist, ucnt, local_order, head_total, head_order, total;
 };
 AttnWs sparse_ws(int B, int H, int N, int block) {
   const size_t bh = static_cast<size_t>(B) * H;
+  const size_t nb = num_blocks(N, block);
+  const size_t groups = (nb + 256 / block - 1) / (256 / block);
   AttnWs w;
-  w.local_order = kWsHeaderBytes;
-  w.head_total = w.local_order + align_up(bh * num_blocks(N, block) * sizeof(int), 256);
+  w.ulist = kWsHeaderBytes;
+  w.ucnt = w.ulist + align_up(bh * groups * nb * sizeof(uint32_t), 256);
+  w.local_order = w.ucnt + align_up(bh * groups * sizeof(int), 256);
+  w.head_total = w.local_order + align_up(bh * groups * sizeof(int), 256);
   w.head_order = w.head_total + align_up(bh * sizeof(unsigned long long), 256);
   w.total = w.head_order + align_up(bh * sizeof(int), 256);
   return w;
@@ -103,13 +110,13 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// [rows, 128] bf16, row stride 256 B; box = 128 rows x 64 columns, 128-byte swizzle.
-bool make_row_map(CUtensorMap* map, const void* base, uint64_t rows) {
+// [rows, 128] bf16, row stride 256 B; box = box_rows rows x 64 columns, 128-byte swizzle.
+bool make_row_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {128, rows};
   cuuint64_t strides[1] = {256};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -165,7 +172,7 @@ fvattn_status attention_fwd(const void* qp, const void* kp, const void* vp, void
   const int nb = num_blocks(N, block);
   if (cudaMemsetAsync(base, 0, kWsHeaderBytes, st) != cudaSuccess) return FVATTN_ERR_CUDA;
 
-  const bool tensor_core = dtype == FVATTN_BF16 && d == 128 && block == 128;
+  const bool tensor_core = dtype == FVATTN_BF16 && d == 128;
   if (!tensor_core) {
     return from_cuda(fvattn::launch_attn_simt(qp, kp, vp, op, lse, sparse ? kv_idx : nullptr,
                                               sparse ? kv_cnt : nullptr, BH, N, d, block,
@@ -173,22 +180,28 @@ fvattn_status attention_fwd(const void* qp, const void* kp, const void* vp, void
   }
   const uint64_t rows = static_cast<uint64_t>(BH) * nb * block;
   CUtensorMap tq, tk, tv;
-  if (!make_row_map(&tq, qp, rows) || !make_row_map(&tk, kp, rows) || !make_row_map(&tv, vp, rows))
+  if (!make_row_map(&tq, qp, rows, 128) || !make_row_map(&tk, kp, rows, block) ||
+      !make_row_map(&tv, vp, rows, block))
     return FVATTN_ERR_CUDA;
   const int sms = device_sm_count();
   if (sms <= 0) return FVATTN_ERR_CUDA;
+  uint32_t* ulist = nullptr;
+  int* ucnt = nullptr;
   int* local_order = nullptr;
   unsigned long long* head_total = nullptr;
   int* head_order = nullptr;
   if (sparse) {
     const AttnWs w = sparse_ws(B, H, N, block);
+    ulist = reinterpret_cast<uint32_t*>(base + w.ulist);
+    ucnt = reinterpret_cast<int*>(base + w.ucnt);
     local_order = reinterpret_cast<int*>(base + w.local_order);
     head_total = reinterpret_cast<unsigned long long*>(base + w.head_total);
     head_order = reinterpret_cast<int*>(base + w.head_order);
   }
   return from_cuda(fvattn::launch_attn_sm100(
-      tq, tk, tv, op, lse, sparse ? kv_idx : nullptr, sparse ? kv_cnt : nullptr, local_order,
-      head_total, head_order, BH, N, nb, scale, &hdr->status, &hdr->counter, sms, st));
+      tq, tk, tv, op, lse, sparse ? kv_idx : nullptr, sparse ? kv_cnt : nullptr, ulist, ucnt,
+      local_order, head_total, head_order, BH, N, nb, block, scale, &hdr->status, &hdr->counter,
+      sms, st));
 }
 
 }  // namespace

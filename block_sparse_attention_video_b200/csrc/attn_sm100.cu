@@ -1,15 +1,23 @@
 // attn_sm100.cu -- block-sparse attention forward on the Blackwell tensor cores
-// (tcgen05 MMA with TMEM accumulators, TMA-fed), bf16 inputs, d = 128, 128-token
-// blocks [FVAttn §2.1: only selected (query block, key block) pairs are
-// evaluated; GSRS §3.2: unselected blocks are skipped in the tiling loop;
-// GSRS §A.1: online softmax, rescaling earlier partial results when the max
-// grows].
+// (tcgen05 MMA with TMEM accumulators, TMA-fed), bf16 inputs, d = 128, blocks of
+// BN = 64 or 128 tokens [FVAttn §2.1: only selected (query block, key block)
+// pairs are evaluated; GSRS §3.2: unselected blocks are skipped in the tiling
+// loop; GSRS §A.1: online softmax, rescaling earlier partial results when the
+// max grows].
 //
-// Work unit = one query block (128 rows) of one (b, h) with its KV block list.
+// Work unit = 256 consecutive query rows of one (b, h), i.e. G = 256/BN query
+// blocks, held as two 128-row Q tiles (slots 0 and 1). The unit walks the
+// UNION of its query blocks' KV lists in ascending block order; each union entry
+// carries a membership bit per query block. Every K/V block of the union is
+// loaded once and feeds both tiles, so adjacent query blocks, whose lists
+// overlap heavily, share their K/V traffic. A tile row whose query block did
+// not select a key block gets P = 0 for it (no exponentials), which leaves its
+// output exactly the softmax over its own selected blocks.
+//
 // Persistent kernel, one CTA per SM, 384 threads (three warpgroups):
-//   warps 0-3  softmax / epilogue of tile slot 0 (thread = query row = TMEM lane)
-//   warps 4-7  softmax / epilogue of tile slot 1
-//   warp  8    TMA producer (one elected thread); also claims work units from a
+//   warps 0-3  softmax / epilogue of slot 0 (thread = query row = TMEM lane)
+//   warps 4-7  softmax / epilogue of slot 1
+//   warp  8    TMA producer (one elected thread); claims work units from a
 //              global counter and publishes them to the other roles
 //   warp  9    TMEM allocator and MMA issuer (one elected thread)
 //   warps 10-11 idle
@@ -18,25 +26,26 @@
 // (2 x 128 x 200 + 128 x 104 = 64,512; per SMSP 2 x 200 + 104 <= 512). Each
 // role ends in its own copy of the teardown so that the compiler allocates
 // registers for each role under its own limit.
-// Each slot walks its own unit's KV list, so the two slots ping-pong on the
-// tensor core: while the softmax warps of one slot exponentiate S, the MMA
-// warp runs the other slot's P.V and next Q.K^T.
 //
+// MMA order per unit: S0(0) S1(0), then for k >= 1: PV0(k-1) S0(k) PV1(k-1)
+// S1(k), and finally PV0(last) PV1(last): the exponentials of one slot overlap
+// the other slot's MMAs.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512).
-// P (bf16, two per 32-bit column) overwrites the first 64 columns of S and is
+// P (bf16, two per 32-bit column) overwrites the first BN/2 columns of S and is
 // the A operand of the P.V MMA straight from TMEM.
-// Shared memory: Q0, Q1 (32 KB each) and a ring of 4 K/V stages (32 KB each),
-// every tile stored as two 128-byte-swizzled halves of 64 columns, as TMA
-// writes them. K-major descriptors for Q and K, an MN-major descriptor for V.
+// Shared memory: Q0, Q1 (32 KB each) and a 128 KB K/V ring (4 x 32 KB stages for
+// BN = 128, 8 x 16 KB for BN = 64), tiles stored as two 128-byte-swizzled halves
+// of 64 columns, as TMA writes them. K-major descriptors for Q and K, MN-major
+// for V.
 //
 // Scheduling [FVAttn §2.2, §3.2: per-head work differs widely across heads]:
-// units are claimed in an order the host prepares (heads by descending work,
-// then each head's query blocks by descending list length), so heavy units
+// units are claimed in an order prepared on the device (heads by descending
+// work, then each head's units by descending union length), so heavy units
 // start first and units that run together share a head's K/V in L2.
 //
 // Softmax: exponent base 2 with scale*log2(e) folded in, P rounded to bf16,
-// fp32 row sums. The running max is only raised (and O rescaled in TMEM) when
-// a block's max exceeds it by more than 8 (a factor 256), which keeps P <= 256.
+// fp32 row sums. The running max is only raised (and O rescaled in TMEM) when a
+// block's max exceeds it by more than 8 (a factor 256), which keeps P <= 256.
 #include <cfloat>
 
 #include "common.cuh"
@@ -45,143 +54,119 @@
 namespace fvattn {
 namespace sm100 {
 
-constexpr int BM = 128;
-constexpr int BN = 128;
 constexpr int HD = 128;
-constexpr int kStages = 4;
-constexpr int kTileBytes = BM * HD * 2;  // 32 KB
-constexpr int kHalfBytes = 128 * 64 * 2; // 16 KB: 128 rows x 128 bytes
+constexpr int kUnitRows = 256;
+constexpr int kQTileBytes = 128 * HD * 2;   // 32 KB
+constexpr int kQHalfBytes = 128 * 128;      // 16 KB: 128 rows x 128 bytes
+constexpr int kRingBytes = 128 * 1024;
 constexpr int kThreads = 384;
 constexpr int kRegsSoftmax = 200;
 constexpr int kRegsControl = 104;
-constexpr uint32_t kIdescQK = umma_idesc_bf16(BM, BN, false);
-constexpr uint32_t kIdescPV = umma_idesc_bf16(BM, HD, true);
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.6931471805599453f;
+
+template <int BN>
+struct Tile {
+  static constexpr int kKVBytes = BN * HD * 2;
+  static constexpr int kKVHalf = BN * 128;
+  static constexpr int kStages = kRingBytes / kKVBytes;
+  static constexpr int kGroup = kUnitRows / BN;   // query blocks per unit
+  static constexpr uint32_t kIdescQK = umma_idesc_bf16(128, BN, false);
+  static constexpr uint32_t kIdescPV = umma_idesc_bf16(128, HD, true);
+};
 
 struct Params {
   int nb;
   int N;
   int npad;
+  int ngroups;
   int total_units;
   float scale_log2;
-  const int* kv_idx;        // nullptr: dense (every block, in order)
-  const int* kv_cnt;
+  const uint32_t* ulist;    // [B*H*ngroups*nb] union entries j | members << 16; nullptr: dense
+  const int* ucnt;          // [B*H*ngroups]
   const int* head_order;    // [B*H] rank -> bh
-  const int* local_order;   // [B*H*nb] (bh, rank) -> query block
+  const int* local_order;   // [B*H*ngroups] (bh, rank) -> group
   __nv_bfloat16* out;
   float* lse;
   int* status;
   unsigned long long* counter;
 };
 
+template <int BN>
 struct __align__(1024) Smem {
-  uint8_t q[2][kTileBytes];
-  uint8_t kv[kStages][kTileBytes];
+  uint8_t q[2][kQTileBytes];
+  uint8_t kv[kRingBytes];
   uint64_t q_full[2];
   uint64_t q_empty[2];
-  uint64_t kv_full[kStages];
-  uint64_t kv_empty[kStages];
+  uint64_t kv_full[Tile<BN>::kStages];
+  uint64_t kv_empty[Tile<BN>::kStages];
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_full[2];
-  uint64_t unit_full[2][2];
-  uint64_t unit_empty[2][2];
+  uint64_t unit_full[2];
+  uint64_t unit_empty[2];
   uint64_t mma_done;
-  int unit_box[2][2];
+  int unit_box[2];
   uint32_t tmem_base;
   int abort_flag;
 };
 
-constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + room to align the base
-
 struct Unit {
-  int bh, i, cnt;
-  const int* list;
+  int bh, grp, cnt;
+  const uint32_t* list;
+  bool slot[2];
 };
 
+template <int BN>
 __device__ __forceinline__ Unit decode_unit(int u, const Params& P) {
+  constexpr int G = Tile<BN>::kGroup;
   Unit x;
   x.bh = 0;
-  x.i = 0;
+  x.grp = 0;
   x.cnt = 0;
   x.list = nullptr;
+  x.slot[0] = x.slot[1] = false;
   if (u < 0 || u >= P.total_units) return x;
-  if (P.kv_idx) {
-    const int r = u / P.nb;
-    const int k = u - r * P.nb;
+  if (P.ulist) {
+    const int r = u / P.ngroups;
+    const int k = u - r * P.ngroups;
     x.bh = __ldg(P.head_order + r);
-    x.i = __ldg(P.local_order + static_cast<size_t>(x.bh) * P.nb + k);
-    const size_t row = static_cast<size_t>(x.bh) * P.nb + x.i;
-    int c = __ldg(P.kv_cnt + row);
-    if (c < 1 || c > P.nb) {
-      record_status(P.status, FVATTN_ERR_INVALID_ARG);
-      c = min(max(c, 1), P.nb);
-    }
-    x.cnt = c;
-    x.list = P.kv_idx + row * P.nb;
+    x.grp = __ldg(P.local_order + static_cast<size_t>(x.bh) * P.ngroups + k);
+    const size_t row = static_cast<size_t>(x.bh) * P.ngroups + x.grp;
+    x.cnt = min(max(__ldg(P.ucnt + row), 1), P.nb);
+    x.list = P.ulist + row * P.nb;
   } else {
-    x.bh = u / P.nb;
-    x.i = u - x.bh * P.nb;
+    x.bh = u / P.ngroups;
+    x.grp = u - x.bh * P.ngroups;
     x.cnt = P.nb;
   }
+  x.slot[0] = x.grp * G < P.nb;
+  x.slot[1] = x.grp * G + G / 2 < P.nb;
   return x;
 }
 
-__device__ __forceinline__ int block_at(const Unit& x, int k, const Params& P) {
-  if (!x.list) return k;
-  int j = __ldg(x.list + k);
-  if (j < 0 || j >= P.nb) {
+template <int BN>
+__device__ __forceinline__ uint32_t entry_at(const Unit& x, int k, const Params& P) {
+  constexpr uint32_t kAll = (1u << Tile<BN>::kGroup) - 1u;
+  if (!x.list) return static_cast<uint32_t>(k) | (kAll << 16);
+  uint32_t e = __ldg(x.list + k);
+  if ((e & 0xFFFFu) >= static_cast<uint32_t>(P.nb)) {
     record_status(P.status, FVATTN_ERR_INVALID_ARG);
-    j = 0;
+    e &= 0xFFFF0000u;
   }
-  return j;
+  return e;
 }
 
-// The op sequence shared by the producer and the MMA issuer. For each slot:
-// S(0); then repeatedly PV(k-1) followed by S(k) (or, at the end of a unit, the
-// next unit's S(0)). Slots alternate step by step.
-template <class GetUnit, class OnS, class OnPV>
-__device__ __forceinline__ bool run_schedule(GetUnit&& get_unit, OnS&& on_s, OnPV&& on_pv) {
-  Unit st[2];
-  int k[2] = {0, 0};
-  bool act[2] = {false, false};
-#pragma unroll
-  for (int X = 0; X < 2; ++X) {
-    if (!get_unit(X, st[X])) return false;
-    act[X] = st[X].cnt > 0;
-    if (act[X]) {
-      if (!on_s(X, st[X], 0)) return false;
-      k[X] = 1;
-    }
-  }
-#pragma unroll 1
-  while (act[0] || act[1]) {
-#pragma unroll
-    for (int X = 0; X < 2; ++X) {
-      if (!act[X]) continue;
-      if (!on_pv(X, st[X], k[X] - 1)) return false;
-      if (k[X] == st[X].cnt) {
-        if (!get_unit(X, st[X])) return false;
-        act[X] = st[X].cnt > 0;
-        if (!act[X]) continue;
-        if (!on_s(X, st[X], 0)) return false;
-        k[X] = 1;
-      } else {
-        if (!on_s(X, st[X], k[X])) return false;
-        ++k[X];
-      }
-    }
-  }
-  return true;
-}
-
+template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const Params P) {
+  using T = Tile<BN>;
+  constexpr int kStages = T::kStages;
+  constexpr int G = T::kGroup;
   extern __shared__ uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>(
+  Smem<BN>& sm = *reinterpret_cast<Smem<BN>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -194,10 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.s_full[X], 1);
       mbar_init(&sm.p_full[X], 4);
       mbar_init(&sm.o_full[X], 1);
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(&sm.unit_full[X][b], 1);
-        mbar_init(&sm.unit_empty[X][b], 5);
-      }
+      mbar_init(&sm.unit_full[X], 1);
+      mbar_init(&sm.unit_empty[X], 9);   // MMA thread + 4 + 4 softmax warps
     }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.kv_full[s], 1);
@@ -227,6 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     asm volatile("barrier.sync 1, %0;" ::"n"(kThreads) : "memory");
     if (warp == 9) {
+      __syncwarp();
       tc_fence_after();
       tmem_dealloc(tmem, 512);
     }
@@ -234,117 +218,123 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp >= 8) {
     regs_dec<kRegsControl>();
-  if (warp == 8) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int it = 0;
+    if (warp == 8 && lane == 0) {
+      // ---------------------------------------------------------- producer
+      int it = 0, un = 0;
       int qn[2] = {0, 0};
-      int un[2] = {0, 0};
-      auto get_unit = [&](int X, Unit& x) -> bool {
-        const int b = un[X] & 1;
-        if (!mbar_wait(&sm.unit_empty[X][b], ((un[X] >> 1) & 1) ^ 1, abort_flag, P.status)) return false;
+      bool ok = true;
+      while (ok) {
+        const int b = un & 1;
+        if (!mbar_wait(&sm.unit_empty[b], ((un >> 1) & 1) ^ 1, abort_flag, P.status)) break;
         int u = static_cast<int>(atomicAdd(P.counter, 1ull));
         if (u >= P.total_units) u = -1;
-        sm.unit_box[X][b] = u;
-        mbar_arrive(&sm.unit_full[X][b]);
-        ++un[X];
-        x = decode_unit(u, P);
-        return true;
-      };
-      auto load_kv = [&](const CUtensorMap* tm, int row) -> bool {
-        const int s = it % kStages;
-        if (!mbar_wait(&sm.kv_empty[s], ((it / kStages) & 1) ^ 1, abort_flag, P.status)) return false;
-        mbar_arrive_expect_tx(&sm.kv_full[s], kTileBytes);
-        tma_load_2d(sm.kv[s], tm, &sm.kv_full[s], 0, row);
-        tma_load_2d(sm.kv[s] + kHalfBytes, tm, &sm.kv_full[s], 64, row);
-        ++it;
-        return true;
-      };
-      auto on_s = [&](int X, const Unit& x, int k) -> bool {
-        if (k == 0) {
-          if (!mbar_wait(&sm.q_empty[X], (qn[X] & 1) ^ 1, abort_flag, P.status)) return false;
-          const int row = x.bh * P.npad + x.i * BM;
-          mbar_arrive_expect_tx(&sm.q_full[X], kTileBytes);
-          tma_load_2d(sm.q[X], &tm_q, &sm.q_full[X], 0, row);
-          tma_load_2d(sm.q[X] + kHalfBytes, &tm_q, &sm.q_full[X], 64, row);
+        sm.unit_box[b] = u;
+        mbar_arrive(&sm.unit_full[b]);
+        ++un;
+        const Unit x = decode_unit<BN>(u, P);
+        if (x.cnt == 0) break;
+        const int row0 = x.bh * P.npad + x.grp * kUnitRows;
+#pragma unroll
+        for (int X = 0; X < 2; ++X) {
+          if (!(X == 0 ? x.slot[0] : x.slot[1])) continue;
+          if (!mbar_wait(&sm.q_empty[X], (qn[X] & 1) ^ 1, abort_flag, P.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&sm.q_full[X], kQTileBytes);
+          tma_load_2d(sm.q[X], &tm_q, &sm.q_full[X], 0, row0 + X * 128);
+          tma_load_2d(sm.q[X] + kQHalfBytes, &tm_q, &sm.q_full[X], 64, row0 + X * 128);
           ++qn[X];
         }
-        return load_kv(&tm_k, x.bh * P.npad + block_at(x, k, P) * BN);
-      };
-      auto on_pv = [&](int X, const Unit& x, int k) -> bool {
-        return load_kv(&tm_v, x.bh * P.npad + block_at(x, k, P) * BN);
-      };
-      run_schedule(get_unit, on_s, on_pv);
+        for (int k = 0; ok && k < x.cnt; ++k) {
+          const int kvrow = x.bh * P.npad + static_cast<int>(entry_at<BN>(x, k, P) & 0xFFFFu) * BN;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {     // K(k) then V(k)
+            const int s = it % kStages;
+            if (!mbar_wait(&sm.kv_empty[s], ((it / kStages) & 1) ^ 1, abort_flag, P.status)) { ok = false; break; }
+            mbar_arrive_expect_tx(&sm.kv_full[s], T::kKVBytes);
+            uint8_t* dst = sm.kv + s * T::kKVBytes;
+            const CUtensorMap* tm = t == 0 ? &tm_k : &tm_v;
+            tma_load_2d(dst, tm, &sm.kv_full[s], 0, kvrow);
+            tma_load_2d(dst + T::kKVHalf, tm, &sm.kv_full[s], 64, kvrow);
+            ++it;
+          }
+        }
+      }
       // Drain: every load this thread armed has landed before the CTA exits.
       for (int o = max(0, it - kStages); o < it; ++o)
         mbar_wait_plain(&sm.kv_full[o % kStages], (o / kStages) & 1);
       for (int X = 0; X < 2; ++X)
         if (qn[X] > 0) mbar_wait_plain(&sm.q_full[X], (qn[X] - 1) & 1);
-    }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int it = 0;
+    } else if (warp == 9 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      int base = 0, un = 0;
       int qn[2] = {0, 0};
       int pn[2] = {0, 0};
-      int un[2] = {0, 0};
       const uint32_t q_addr[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
-      auto get_unit = [&](int X, Unit& x) -> bool {
-        const int b = un[X] & 1;
-        if (!mbar_wait(&sm.unit_full[X][b], (un[X] >> 1) & 1, abort_flag, P.status)) return false;
-        const int u = *reinterpret_cast<volatile int*>(&sm.unit_box[X][b]);
-        mbar_arrive(&sm.unit_empty[X][b]);
-        ++un[X];
-        x = decode_unit(u, P);
-        return true;
-      };
-      auto on_s = [&](int X, const Unit& x, int k) -> bool {
-        if (k == 0) {
-          if (!mbar_wait(&sm.q_full[X], qn[X] & 1, abort_flag, P.status)) return false;
-          ++qn[X];
-        }
-        const int s = it % kStages;
-        if (!mbar_wait(&sm.kv_full[s], (it / kStages) & 1, abort_flag, P.status)) return false;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sm.kv[s]);
-        const uint32_t d_tmem = tmem + X * 128;
+      const uint32_t kv_addr = smem_u32(sm.kv);
+      bool ok = true;
+      while (ok) {
+        const int b = un & 1;
+        if (!mbar_wait(&sm.unit_full[b], (un >> 1) & 1, abort_flag, P.status)) break;
+        const int u = *reinterpret_cast<volatile int*>(&sm.unit_box[b]);
+        mbar_arrive(&sm.unit_empty[b]);
+        ++un;
+        const Unit x = decode_unit<BN>(u, P);
+        if (x.cnt == 0) break;
+        const int cnt = x.cnt;
+        auto kv_ready = [&](int o) -> bool {
+          return mbar_wait(&sm.kv_full[o % kStages], (o / kStages) & 1, abort_flag, P.status);
+        };
+        auto s_op = [&](int X, int k) -> bool {   // S_X = Q_X K(k)^T, K(k) already waited on
+          if (k == 0) {
+            if (!mbar_wait(&sm.q_full[X], qn[X] & 1, abort_flag, P.status)) return false;
+            ++qn[X];
+          }
+          tc_fence_after();
+          const uint32_t ka = kv_addr + ((base + 2 * k) % kStages) * T::kKVBytes;
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          umma_ss(d_tmem, umma_desc_sw128(q_addr[X] + off, 16, 1024),
-                  umma_desc_sw128(k_addr + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(&sm.kv_empty[s]);
-        umma_commit(&sm.s_full[X]);
-        if (k == x.cnt - 1) umma_commit(&sm.q_empty[X]);
-        ++it;
-        return true;
-      };
-      auto on_pv = [&](int X, const Unit& x, int k) -> bool {
-        if (!mbar_wait(&sm.p_full[X], pn[X] & 1, abort_flag, P.status)) return false;
-        ++pn[X];
-        const int s = it % kStages;
-        if (!mbar_wait(&sm.kv_full[s], (it / kStages) & 1, abort_flag, P.status)) return false;
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(sm.kv[s]);
-        const uint32_t p_tmem = tmem + X * 128;
-        const uint32_t o_tmem = tmem + 256 + X * 128;
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            umma_ss(tmem + X * 128,
+                    umma_desc_sw128(q_addr[X] + (kk >> 2) * kQHalfBytes + (kk & 3) * 32, 16, 1024),
+                    umma_desc_sw128(ka + (kk >> 2) * T::kKVHalf + (kk & 3) * 32, 16, 1024),
+                    T::kIdescQK, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&sm.s_full[X]);
+          if (k == cnt - 1) umma_commit(&sm.q_empty[X]);
+          return true;
+        };
+        auto pv_op = [&](int X, int k) -> bool {  // O_X += P_X V(k), V(k) already waited on
+          if (!mbar_wait(&sm.p_full[X], pn[X] & 1, abort_flag, P.status)) return false;
+          ++pn[X];
+          tc_fence_after();
+          const uint32_t va = kv_addr + ((base + 2 * k + 1) % kStages) * T::kKVBytes;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          umma_ts(o_tmem, p_tmem + kk * 8, umma_desc_sw128(v_addr + kk * 2048, kHalfBytes, 1024),
-                  kIdescPV, (k > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            umma_ts(tmem + 256 + X * 128, tmem + X * 128 + kk * 8,
+                    umma_desc_sw128(va + kk * 2048, T::kKVHalf, 1024), T::kIdescPV,
+                    (k > 0 || kk > 0) ? 1u : 0u);
+          }
+          if (k == cnt - 1) umma_commit(&sm.o_full[X]);
+          return true;
+        };
+        const bool two = x.slot[1];
+        ok = kv_ready(base) && s_op(0, 0) && (!two || s_op(1, 0));
+        if (ok) umma_commit(&sm.kv_empty[base % kStages]);
+        for (int k = 1; ok && k < cnt; ++k) {
+          ok = kv_ready(base + 2 * k - 1) && pv_op(0, k - 1) && kv_ready(base + 2 * k) && s_op(0, k) &&
+               (!two || pv_op(1, k - 1));
+          if (!ok) break;
+          umma_commit(&sm.kv_empty[(base + 2 * k - 1) % kStages]);
+          ok = !two || s_op(1, k);
+          if (!ok) break;
+          umma_commit(&sm.kv_empty[(base + 2 * k) % kStages]);
         }
-        umma_commit(&sm.kv_empty[s]);
-        if (k == x.cnt - 1) umma_commit(&sm.o_full[X]);
-        ++it;
-        return true;
-      };
-      run_schedule(get_unit, on_s, on_pv);
+        if (ok) ok = kv_ready(base + 2 * cnt - 1) && pv_op(0, cnt - 1) && (!two || pv_op(1, cnt - 1));
+        if (ok) umma_commit(&sm.kv_empty[(base + 2 * cnt - 1) % kStages]);
+        base += 2 * cnt;
+      }
       // Drain: every MMA this thread issued has completed before TMEM is freed.
       umma_commit(&sm.mma_done);
       mbar_wait_plain(&sm.mma_done, 0);
     }
-  }
     teardown();
     return;
   }
@@ -352,9 +342,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   regs_inc<kRegsSoftmax>();
   {
     // ------------------------------------------------------------ softmax / epilogue
+    constexpr int NC = BN / 32;          // 32-column chunks of S
     const int X = warp >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
+    const int qb = (X * 128 + row) / BN;  // query block of this row within the unit
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tS = tmem + lane_off + X * 128;
     const uint32_t tO = tmem + lane_off + 256 + X * 128;
@@ -364,72 +356,87 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
     while (true) {
       const int b = n & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.unit_full[X][b], (n >> 1) & 1, abort_flag, P.status))) break;
-      const int u = *reinterpret_cast<volatile int*>(&sm.unit_box[X][b]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.unit_full[b], (n >> 1) & 1, abort_flag, P.status))) break;
+      const int u = *reinterpret_cast<volatile int*>(&sm.unit_box[b]);
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.unit_empty[X][b]);
+      if (lane == 0) mbar_arrive(&sm.unit_empty[b]);
       ++n;
-      const Unit x = decode_unit(u, P);
+      const Unit x = decode_unit<BN>(u, P);
       if (x.cnt == 0) break;
+      if (!(X == 0 ? x.slot[0] : x.slot[1])) continue;
       float m_run = -FLT_MAX;
       float l_run = 0.f;
+      bool have = false;
       bool ok = true;
 #pragma unroll 1
       for (int k = 0; k < x.cnt; ++k) {
         if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[X], sn & 1, abort_flag, P.status))) { ok = false; break; }
         ++sn;
         tc_fence_after();
-        uint32_t s[4][32];
-        tmem_ld32(tS + 0, s[0]);
-        tmem_ld32(tS + 32, s[1]);
-        tmem_ld32(tS + 64, s[2]);
-        tmem_ld32(tS + 96, s[3]);
-        tmem_wait_ld();
-        const int j = block_at(x, k, P);
-        if (j == P.nb - 1 && tail < BN) {
+        const uint32_t e = entry_at<BN>(x, k, P);
+        if ((e >> (16 + qb)) & 1u) {
+          uint32_t s[NC][32];
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < NC; ++c) tmem_ld32(tS + c * 32, s[c]);
+          tmem_wait_ld();
+          if (static_cast<int>(e & 0xFFFFu) == P.nb - 1 && tail < BN) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (c * 32 + e >= tail) s[c][e] = __float_as_uint(-INFINITY);
-        }
-        float mx = -FLT_MAX;
+            for (int c = 0; c < NC; ++c)
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+              for (int i = 0; i < 32; ++i)
+                if (c * 32 + i >= tail) s[c][i] = __float_as_uint(-INFINITY);
+          }
+          float mx = -FLT_MAX;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(s[c][e]));
-        const float m_new = mx * sl2;
-        if (k == 0) {
-          m_run = m_new;
-        } else if (m_new > m_run + kRescaleThreshold) {
-          const float f = ex2_approx(m_run - m_new);
-          l_run *= f;
+          for (int c = 0; c < NC; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(s[c][i]));
+          const float m_new = mx * sl2;
+          if (!have) {
+            m_run = m_new;
+            have = true;
+          } else {
+            // The decision is per row but tcgen05.ld/st are warp-collective: when
+            // any row of the warp needs a larger max, the whole warp rescales,
+            // rows that do not need it with factor 1.
+            const bool need = m_new > m_run + kRescaleThreshold;
+            if (__any_sync(0xffffffffu, need)) {
+              const float f = need ? ex2_approx(m_run - m_new) : 1.f;
+              l_run *= f;
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + c * 32, o);
-            tmem_wait_ld();
+              for (int c = 0; c < 4; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tO + c * 32, o);
+                tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-            tmem_st32(tO + c * 32, o);
+                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+                tmem_st32(tO + c * 32, o);
+              }
+              tmem_wait_st();
+              if (need) m_run = m_new;
+            }
           }
-          tmem_wait_st();
-          m_run = m_new;
-        }
-        float lsum = 0.f;
+          float lsum = 0.f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
+          for (int c = 0; c < NC; ++c) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(s[c][2 * e]), sl2, -m_run));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(s[c][2 * e + 1]), sl2, -m_run));
-            lsum += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
+            for (int i = 0; i < 16; ++i) {
+              const float p0 = ex2_approx(fmaf(__uint_as_float(s[c][2 * i]), sl2, -m_run));
+              const float p1 = ex2_approx(fmaf(__uint_as_float(s[c][2 * i + 1]), sl2, -m_run));
+              lsum += p0 + p1;
+              pk[i] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(tS + c * 16, pk);
           }
-          tmem_st16(tS + c * 16, pk);
+          l_run += lsum;
+        } else {
+          uint32_t z[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) z[i] = 0u;
+#pragma unroll
+          for (int c = 0; c < NC; ++c) tmem_st16(tS + c * 16, z);
         }
-        l_run += lsum;
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -439,8 +446,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_full[X], on & 1, abort_flag, P.status))) break;
       ++on;
       tc_fence_after();
-      const float inv_l = 1.f / l_run;
-      const size_t grow = static_cast<size_t>(x.bh) * P.npad + static_cast<size_t>(x.i) * BM + row;
+      // Rows past the head's last block (the second half of a 64-token-block
+      // tile at the end of a head) are not stored; the TMEM loads stay
+      // warp-collective.
+      const int qrow = x.grp * kUnitRows + X * 128 + row;   // row within the head
+      const bool store = qrow < P.npad;
+      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      const size_t grow = static_cast<size_t>(x.bh) * P.npad + qrow;
       uint4* orow = reinterpret_cast<uint4*>(P.out + grow * HD);
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
@@ -449,25 +461,86 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+        for (int i = 0; i < 16; ++i)
+          w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+        if (store) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          orow[c * 4 + e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          for (int i = 0; i < 4; ++i)
+            orow[c * 4 + i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
       }
-      if (P.lse) P.lse[grow] = (m_run + __log2f(l_run)) * kLn2;
+      if (store && P.lse) P.lse[grow] = (m_run + __log2f(l_run)) * kLn2;
       tc_fence_before();
     }
   }
-
   teardown();
 }
 
 }  // namespace sm100
 
 // ---------------------------------------------------------------- work order
-// Within each head: query blocks by descending list length (ties: lower index).
-// Per head: total work. Then heads by descending total (ties: lower index).
+// plan_union_kernel: per (b, h) and group of G consecutive query blocks, the
+// ascending union of their KV lists with one membership bit per query block
+// (bitmaps in shared memory; out-of-range entries are dropped and recorded).
+template <int G>
+__global__ void __launch_bounds__(256)
+    plan_union_kernel(const int* __restrict__ kv_idx, const int* __restrict__ kv_cnt, int nb,
+                      int ngroups, uint32_t* __restrict__ ulist, int* __restrict__ ucnt,
+                      int* status) {
+  __shared__ uint32_t bm[G][128];
+  __shared__ int base[129];
+  const int grp = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int nwords = (nb + 31) >> 5;
+  for (int t = threadIdx.x; t < G * 128; t += blockDim.x) bm[t / 128][t % 128] = 0u;
+  __syncthreads();
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const int i = grp * G + g;
+    if (i >= nb) break;
+    const size_t row = static_cast<size_t>(bh) * nb + i;
+    int c = kv_cnt[row];
+    if (c < 1 || c > nb) {
+      if (threadIdx.x == 0) record_status(status, FVATTN_ERR_INVALID_ARG);
+      c = min(max(c, 1), nb);
+    }
+    for (int t = threadIdx.x; t < c; t += blockDim.x) {
+      const int j = kv_idx[row * nb + t];
+      if (j >= 0 && j < nb) atomicOr(&bm[g][j >> 5], 1u << (j & 31));
+      else record_status(status, FVATTN_ERR_INVALID_ARG);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < nwords) {
+    uint32_t m = 0u;
+#pragma unroll
+    for (int g = 0; g < G; ++g) m |= bm[g][threadIdx.x];
+    base[threadIdx.x + 1] = __popc(m);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    base[0] = 0;
+    for (int w = 1; w <= nwords; ++w) base[w] += base[w - 1];
+    ucnt[static_cast<size_t>(bh) * ngroups + grp] = base[nwords];
+  }
+  __syncthreads();
+  if (threadIdx.x < nwords) {
+    const int w = threadIdx.x;
+    uint32_t m = 0u;
+#pragma unroll
+    for (int g = 0; g < G; ++g) m |= bm[g][w];
+    uint32_t* out = ulist + (static_cast<size_t>(bh) * ngroups + grp) * nb + base[w];
+    while (m) {
+      const int bit = __ffs(m) - 1;
+      m &= m - 1u;
+      uint32_t members = 0u;
+#pragma unroll
+      for (int g = 0; g < G; ++g) members |= ((bm[g][w] >> bit) & 1u) << g;
+      *out++ = static_cast<uint32_t>(w * 32 + bit) | (members << 16);
+    }
+  }
+}
+
 __device__ __forceinline__ void bitonic_desc_u32(uint32_t* a, int n) {
   for (int size = 2; size <= n; size <<= 1)
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
@@ -498,18 +571,19 @@ __device__ __forceinline__ void bitonic_desc_u64(unsigned long long* a, int n) {
   __syncthreads();
 }
 
+// Within each head: units by descending union length (ties: lower index); the head's total.
 __global__ void __launch_bounds__(1024)
-    plan_heads_kernel(const int* __restrict__ kv_cnt, int nb, int* __restrict__ local_order,
+    plan_heads_kernel(const int* __restrict__ ucnt, int ngroups, int* __restrict__ local_order,
                       unsigned long long* __restrict__ head_total) {
   __shared__ uint32_t keys[4096];
   __shared__ unsigned long long red[32];
   const int bh = blockIdx.x;
   int n2 = 1;
-  while (n2 < nb) n2 <<= 1;
+  while (n2 < ngroups) n2 <<= 1;
   unsigned long long part = 0;
   for (int i = threadIdx.x; i < n2; i += blockDim.x) {
-    if (i < nb) {
-      const int c = min(max(kv_cnt[static_cast<size_t>(bh) * nb + i], 1), nb);
+    if (i < ngroups) {
+      const int c = ucnt[static_cast<size_t>(bh) * ngroups + i];
       keys[i] = (static_cast<uint32_t>(c) << 16) | static_cast<uint32_t>(0xFFFF - i);
       part += static_cast<unsigned long long>(c);
     } else {
@@ -521,11 +595,11 @@ __global__ void __launch_bounds__(1024)
   bitonic_desc_u32(keys, n2);
   if (threadIdx.x == 0) {
     unsigned long long t = 0;
-    for (int w = 0; w < (blockDim.x + 31) / 32; ++w) t += red[w];
+    for (int w = 0; w < static_cast<int>(blockDim.x + 31) / 32; ++w) t += red[w];
     head_total[bh] = t;
   }
-  for (int r = threadIdx.x; r < nb; r += blockDim.x)
-    local_order[static_cast<size_t>(bh) * nb + r] = 0xFFFF - static_cast<int>(keys[r] & 0xFFFFu);
+  for (int r = threadIdx.x; r < ngroups; r += blockDim.x)
+    local_order[static_cast<size_t>(bh) * ngroups + r] = 0xFFFF - static_cast<int>(keys[r] & 0xFFFFu);
 }
 
 __global__ void __launch_bounds__(1024)
@@ -542,15 +616,34 @@ __global__ void __launch_bounds__(1024)
 }
 
 // ---------------------------------------------------------------- launcher
-size_t attn_sm100_smem_bytes() { return sm100::kSmemBytes; }
+template <int BN>
+static cudaError_t launch_bn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const sm100::Params& P, int num_sms, cudaStream_t st) {
+  const size_t smem = sizeof(sm100::Smem<BN>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(sm100::attn_fwd_sm100_kernel<BN>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int grid = max(1, min(num_sms, P.total_units));
+  sm100::attn_fwd_sm100_kernel<BN><<<grid, sm100::kThreads, smem, st>>>(tq, tk, tv, P);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_attn_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                               void* out, float* lse, const int* kv_idx, const int* kv_cnt,
-                              int* local_order, unsigned long long* head_total, int* head_order,
-                              int BH, int N, int nb, float scale, int* status,
+                              uint32_t* ulist, int* ucnt, int* local_order,
+                              unsigned long long* head_total, int* head_order, int BH, int N,
+                              int nb, int bs, float scale, int* status,
                               unsigned long long* counter, int num_sms, cudaStream_t st) {
+  const int G = sm100::kUnitRows / bs;
+  const int ngroups = (nb + G - 1) / G;
   if (kv_idx) {
-    plan_heads_kernel<<<BH, 1024, 0, st>>>(kv_cnt, nb, local_order, head_total);
+    const dim3 g1(ngroups, BH);
+    if (G == 2)
+      plan_union_kernel<2><<<g1, 256, 0, st>>>(kv_idx, kv_cnt, nb, ngroups, ulist, ucnt, status);
+    else
+      plan_union_kernel<4><<<g1, 256, 0, st>>>(kv_idx, kv_cnt, nb, ngroups, ulist, ucnt, status);
+    plan_heads_kernel<<<BH, 1024, 0, st>>>(ucnt, ngroups, local_order, head_total);
     plan_rank_kernel<<<1, 1024, 0, st>>>(head_total, BH, head_order);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -558,24 +651,19 @@ cudaError_t launch_attn_sm100(const CUtensorMap& tq, const CUtensorMap& tk, cons
   sm100::Params P;
   P.nb = nb;
   P.N = N;
-  P.npad = nb * sm100::BM;
-  P.total_units = BH * nb;
+  P.npad = nb * bs;
+  P.ngroups = ngroups;
+  P.total_units = BH * ngroups;
   P.scale_log2 = scale * 1.4426950408889634f;
-  P.kv_idx = kv_idx;
-  P.kv_cnt = kv_cnt;
+  P.ulist = kv_idx ? ulist : nullptr;
+  P.ucnt = ucnt;
   P.head_order = head_order;
   P.local_order = local_order;
   P.out = static_cast<__nv_bfloat16*>(out);
   P.lse = lse;
   P.status = status;
   P.counter = counter;
-  cudaError_t e = cudaFuncSetAttribute(sm100::attn_fwd_sm100_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(sm100::kSmemBytes));
-  if (e != cudaSuccess) return e;
-  const int grid = max(1, min(num_sms, P.total_units));
-  sm100::attn_fwd_sm100_kernel<<<grid, sm100::kThreads, sm100::kSmemBytes, st>>>(tq, tk, tv, P);
-  return cudaGetLastError();
+  return bs == 64 ? launch_bn<64>(tq, tk, tv, P, num_sms, st) : launch_bn<128>(tq, tk, tv, P, num_sms, st);
 }
 
 }  // namespace fvattn

@@ -68,7 +68,7 @@ typedef enum {
 } fvattn_status;
 
 typedef enum {
-  FVATTN_BF16 = 0, /* tensor-core path (d = 128, block = 128) and SIMT path */
+  FVATTN_BF16 = 0, /* tensor-core path (d = 128) and SIMT path (d = 64)     */
   FVATTN_FP32 = 1  /* SIMT path only (fp32 arithmetic throughout)           */
 } fvattn_dtype;
 
@@ -135,9 +135,11 @@ FVATTN_API fvattn_status fvattn_route(const void* q, const void* k, int B, int H
  * over the attended keys (NULL to skip). Rows >= N of op and lse are written
  * but carry no meaning. kv_idx/kv_cnt as produced by fvattn_route (any order
  * of entries within a row is accepted). scale > 0 (1/sqrt(d) is the usual).
- * BF16 with d == 128 and block == 128 runs the tcgen05/TMEM tensor-core kernel
- * (bf16 MMA, fp32 accumulation and softmax, P rounded to bf16); other shapes
- * and FP32 run the SIMT kernel (fp32 throughout).
+ * BF16 with d == 128 (block 64 or 128) runs the tcgen05/TMEM tensor-core
+ * kernel (bf16 MMA, fp32 accumulation and softmax, P rounded to bf16); it
+ * processes 256 query rows at a time over the union of their blocks' lists,
+ * masking each row to its own block's list. d == 64 and FP32 run the SIMT
+ * kernel (fp32 throughout).
  * Workspace: fvattn_workspace_bytes(FVATTN_OP_SPARSE_FWD, ...). */
 FVATTN_API fvattn_status fvattn_sparse_fwd(const void* qp, const void* kp, const void* vp,
                                 void* op, float* lse, const int32_t* kv_idx,

@@ -63,6 +63,10 @@ ODD128 = S.Workload("odd-grid-128", 2, 3, 128, "bf16", (3, 10, 14), (2, 8, 8), 1
 SINGLE = S.Workload("single-block", 1, 2, 128, "bf16", (1, 8, 10), (1, 8, 8), 128, 0.9, 1, seed=13)
 TINY_BF16 = S.Workload("tiny-bf16-d128", 1, 2, 128, "bf16", (4, 16, 16), (1, 8, 16), 128, 0.9, 1,
                        seed=14, gen="gauss", peaky_head=1, peaky_scale=3.0)
+# Large logits make the running max jump often, exercising the O rescale in TMEM.
+PEAKY = S.Workload("peaky-rescale", 1, 3, 128, "bf16", (4, 16, 24), (1, 8, 16), 128, 0.97, 2,
+                   seed=15, gen="gauss", peaky_head=2, peaky_scale=8.0)
+BS64 = S.Workload("bs64-d128", 2, 2, 128, "bf16", (5, 12, 20), (1, 8, 8), 64, 0.8, 3, seed=16)
 
 
 # ----------------------------------------------------------------- permutation
@@ -154,7 +158,7 @@ def _sample_blocks(w, nb, cnt=None, per_head=6, seed=0):
     return out
 
 
-@pytest.mark.parametrize("w", [S.WORKLOADS["tiny"], ODD, ODD128, SINGLE, TINY_BF16],
+@pytest.mark.parametrize("w", [S.WORKLOADS["tiny"], ODD, ODD128, SINGLE, TINY_BF16, PEAKY, BS64],
                          ids=lambda w: w.name)
 def test_sparse_and_dense_attention_all_blocks(w):
     q, k, v = S.make_qkv(w, device="cuda")
