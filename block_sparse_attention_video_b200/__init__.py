@@ -4,11 +4,11 @@ Every step of the attention path runs in the library's CUDA kernels; this
 module turns torch tensors into pointers and sizes, passes the current CUDA
 stream, and raises on a non-OK status. It never computes on the CPU and has no
 fallback: importing it fails loudly if the library has not been built
-(``python -m block_sparse_attention_video_b200.build_lib``).
+(``python block_sparse_attention_video_b200/build_lib.py``).
 
 Entry points carry the C names: ``fvattn_permute``, ``fvattn_route``,
-``fvattn_sparse_fwd``, ``fvattn_dense_fwd``, ``fvattn_workspace_bytes``,
-``fvattn_workspace_status``. ``FVAttnPath`` strings them into the full per-call
+``fvattn_route_noalloc``, ``fvattn_sparse_fwd``, ``fvattn_dense_fwd``,
+``fvattn_workspace_bytes``, ``fvattn_workspace_status``. ``FVAttnPath`` strings them into the full per-call
 path (route -> permute V -> block-sparse attention -> inverse permute) over
 buffers it allocates once with torch.
 """
@@ -27,7 +27,7 @@ LIB_PATH = os.path.join(_HERE, "libfvattn.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"{LIB_PATH} is missing: build it with "
-        "`python -m block_sparse_attention_video_b200.build_lib` (nvcc, sm_100a)")
+        "`python block_sparse_attention_video_b200/build_lib.py` (nvcc, sm_100a)")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -45,8 +45,8 @@ FVATTN_OP_ROUTE = 0
 FVATTN_OP_SPARSE_FWD = 1
 FVATTN_OP_DENSE_FWD = 2
 
-EXPORTED = ("fvattn_workspace_bytes", "fvattn_permute", "fvattn_route", "fvattn_sparse_fwd",
-            "fvattn_dense_fwd", "fvattn_workspace_status", "fvattn_status_string")
+EXPORTED = ("fvattn_workspace_bytes", "fvattn_permute", "fvattn_route", "fvattn_route_noalloc",
+            "fvattn_sparse_fwd", "fvattn_dense_fwd", "fvattn_workspace_status", "fvattn_status_string")
 
 
 class Grid(ctypes.Structure):
@@ -78,6 +78,10 @@ _lib.fvattn_route.argtypes = [_c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_i
                               ctypes.POINTER(Grid), _c_float, _c_int, _c_void_p, _c_void_p,
                               _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_void_p]
 _lib.fvattn_route.restype = _c_int
+_lib.fvattn_route_noalloc.argtypes = [_c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                      ctypes.POINTER(Grid), _c_float, _c_int, _c_void_p, _c_void_p,
+                                      _c_void_p, _c_void_p, _c_void_p, _c_void_p]
+_lib.fvattn_route_noalloc.restype = _c_int
 _lib.fvattn_sparse_fwd.argtypes = [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                                    _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
                                    _c_int, _c_float, _c_void_p, _c_size_t, _c_void_p]
@@ -153,6 +157,20 @@ def fvattn_route(q, k, grid: Grid, p: float, k_min: int, kv_idx, kv_cnt, head_wo
                              _ptr(kv_cnt), _ptr(head_work), _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream(stream)),
            "fvattn_route")
+    return kv_idx, kv_cnt, head_work
+
+
+def fvattn_route_noalloc(q, k, grid: Grid, p: float, k_min: int, kv_idx, kv_cnt, head_work,
+                         qp_out=None, kp_out=None, stream=None):
+    """fvattn_route without a workspace, for callers that cannot allocate device
+    memory where they route; the library's static 32 MiB device scratch is used
+    instead (calls that overlap on the GPU race on it)."""
+    _need_cuda(q, k, kv_idx, kv_cnt, head_work, qp_out, kp_out)
+    B, H, N, d = q.shape
+    _check(_lib.fvattn_route_noalloc(_ptr(q), _ptr(k), B, H, N, d, _dtype_code(q), ctypes.byref(grid),
+                                     float(p), int(k_min), _ptr(qp_out), _ptr(kp_out), _ptr(kv_idx),
+                                     _ptr(kv_cnt), _ptr(head_work), _stream(stream)),
+           "fvattn_route_noalloc")
     return kv_idx, kv_cnt, head_work
 
 

@@ -1,6 +1,9 @@
 """Build libfvattn.so in-tree for sm_100a with nvcc.
 
-    python -m block_sparse_attention_video_b200.build_lib [--force] [--verbose]
+    python block_sparse_attention_video_b200/build_lib.py [--force] [--verbose]
+
+(Run it by path: importing it as a submodule would import the package, which
+loads the library it is about to build.)
 
 Each .cu file under csrc/ compiles to an object in _build/ (in parallel, only
 when its sources changed); the objects link into
@@ -24,7 +27,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfvattn.so")
 HEADER = os.path.join(ROOT, "include", "fvattn.h")
-SOURCES = ["api.cu", "permute.cu", "route.cu", "attn_simt.cu", "attn_sm100.cu"]
+SOURCES = ["api.cu", "permute.cu", "route.cu", "attn_simt.cu", "attn_sm100.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "-Xptxas", "-warn-spills", f"-I{os.path.join(ROOT, 'include')}"]

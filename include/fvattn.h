@@ -127,6 +127,23 @@ FVATTN_API fvattn_status fvattn_route(const void* q, const void* k, int B, int H
                            int32_t* kv_cnt, int64_t* head_work, void* workspace,
                            size_t workspace_bytes, void* stream);
 
+/* fvattn_route for callers that cannot allocate device memory at the call
+ * site (an engine plugin with no scratch buffer to offer, or a hot loop where
+ * cudaMalloc would synchronize the device). The pages have no counterpart to
+ * this call; it exists only for how the library is embedded.
+ * Same arguments and results as fvattn_route, minus the workspace: the scratch
+ * is a library-owned static device array of 32 MiB that every GPU loading the
+ * library keeps until exit. Sizes whose route workspace exceeds 32 MiB return
+ * FVATTN_ERR_WORKSPACE and launch nothing. All calls on a device share the
+ * array, so calls that overlap on the GPU race; the first call on each device
+ * looks up the array's address (do it before any stream capture). Nothing is
+ * allocated. Kernel-side status words are not reported by this variant. */
+FVATTN_API fvattn_status fvattn_route_noalloc(const void* q, const void* k, int B, int H, int N,
+                                              int d, fvattn_dtype dtype, const fvattn_grid* grid,
+                                              float p, int k_min, void* qp_out, void* kp_out,
+                                              int32_t* kv_idx, int32_t* kv_cnt,
+                                              int64_t* head_work, void* stream);
+
 /* Block-sparse attention forward [FVAttn §2.1; GSRS §3.2, §A.1].
  * qp, kp, vp [B,H,Npad,d] in tile order (pad rows zero), op [B,H,Npad,d] out.
  * For every query token of query block i: softmax over the valid keys (index
