@@ -22,8 +22,8 @@
 //   warp  9    TMEM allocator and MMA issuer (one elected thread)
 //   warps 10-11 idle
 // The block launches with 168 registers per thread (384 x 168 = 64,512); the
-// third warpgroup drops to 104 and the two softmax warpgroups rise to 200
-// (2 x 128 x 200 + 128 x 104 = 64,512; per SMSP 2 x 200 + 104 <= 512). Each
+// third warpgroup drops to 128 and the two softmax warpgroups rise to 184
+// (2 x 128 x 184 + 128 x 128 = 63,488 <= 64,512; per SMSP 2 x 184 + 128 <= 512). Each
 // role ends in its own copy of the teardown so that the compiler allocates
 // registers for each role under its own limit.
 //
@@ -60,10 +60,16 @@ constexpr int kQTileBytes = 128 * HD * 2;   // 32 KB
 constexpr int kQHalfBytes = 128 * 128;      // 16 KB: 128 rows x 128 bytes
 constexpr int kRingBytes = 128 * 1024;
 constexpr int kThreads = 384;
-constexpr int kRegsSoftmax = 200;
-constexpr int kRegsControl = 104;
+constexpr int kRegsSoftmax = 184;
+constexpr int kRegsControl = 128;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.6931471805599453f;
+// One in kPolyEvery exponential pairs runs on the FMA pipe (exp2_poly3), the
+// rest on MUFU; 0 keeps every exponential on MUFU.
+#ifndef FVATTN_POLY_EVERY
+#define FVATTN_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = FVATTN_POLY_EVERY;
 
 template <int BN>
 struct Tile {
@@ -101,7 +107,7 @@ struct __align__(1024) Smem {
   uint64_t kv_full[Tile<BN>::kStages];
   uint64_t kv_empty[Tile<BN>::kStages];
   uint64_t s_full[2];
-  uint64_t p_full[2];
+  uint64_t p_full[2][2];   // [slot][half of P]
   uint64_t o_full[2];
   uint64_t unit_full[2];
   uint64_t unit_empty[2];
@@ -164,7 +170,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                           const __grid_constant__ CUtensorMap tm_v, const Params P) {
   using T = Tile<BN>;
   constexpr int kStages = T::kStages;
-  constexpr int G = T::kGroup;
   extern __shared__ uint8_t smem_raw[];
   Smem<BN>& sm = *reinterpret_cast<Smem<BN>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -177,7 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.q_full[X], 1);
       mbar_init(&sm.q_empty[X], 1);
       mbar_init(&sm.s_full[X], 1);
-      mbar_init(&sm.p_full[X], 4);
+      mbar_init(&sm.p_full[X][0], 4);
+      mbar_init(&sm.p_full[X][1], 4);
       mbar_init(&sm.o_full[X], 1);
       mbar_init(&sm.unit_full[X], 1);
       mbar_init(&sm.unit_empty[X], 9);   // MMA thread + 4 + 4 softmax warps
@@ -302,16 +308,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         };
         auto pv_op = [&](int X, int k) -> bool {  // O_X += P_X V(k), V(k) already waited on
-          if (!mbar_wait(&sm.p_full[X], pn[X] & 1, abort_flag, P.status)) return false;
-          ++pn[X];
-          tc_fence_after();
+          // P arrives in two halves (key columns [0, BN/2) and [BN/2, BN)); the
+          // first half's MMAs run while the softmax warps finish the second.
           const uint32_t va = kv_addr + ((base + 2 * k + 1) % kStages) * T::kKVBytes;
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            umma_ts(tmem + 256 + X * 128, tmem + X * 128 + kk * 8,
-                    umma_desc_sw128(va + kk * 2048, T::kKVHalf, 1024), T::kIdescPV,
-                    (k > 0 || kk > 0) ? 1u : 0u);
+          for (int h = 0; h < 2; ++h) {
+            if (!mbar_wait(&sm.p_full[X][h], pn[X] & 1, abort_flag, P.status)) return false;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = h * (BN / 32); kk < (h + 1) * (BN / 32); ++kk) {
+              umma_ts(tmem + 256 + X * 128, tmem + X * 128 + kk * 8,
+                      umma_desc_sw128(va + kk * 2048, T::kKVHalf, 1024), T::kIdescPV,
+                      (k > 0 || kk > 0) ? 1u : 0u);
+            }
           }
+          ++pn[X];
           if (k == cnt - 1) umma_commit(&sm.o_full[X]);
           return true;
         };
@@ -368,12 +379,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       float l_run = 0.f;
       bool have = false;
       bool ok = true;
+      uint32_t e_next = entry_at<BN>(x, 0, P);
 #pragma unroll 1
       for (int k = 0; k < x.cnt; ++k) {
         if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[X], sn & 1, abort_flag, P.status))) { ok = false; break; }
         ++sn;
         tc_fence_after();
-        const uint32_t e = entry_at<BN>(x, k, P);
+        const uint32_t e = e_next;
+        if (k + 1 < x.cnt) e_next = entry_at<BN>(x, k + 1, P);   // hide the list read behind this block
         if ((e >> (16 + qb)) & 1u) {
           uint32_t s[NC][32];
 #pragma unroll
@@ -386,11 +399,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int i = 0; i < 32; ++i)
                 if (c * 32 + i >= tail) s[c][i] = __float_as_uint(-INFINITY);
           }
-          float mx = -FLT_MAX;
+          // Row max: 8 independent chains of 3-input max (exact in any order).
+          float mx8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx8[i] = -FLT_MAX;
 #pragma unroll
           for (int c = 0; c < NC; ++c)
 #pragma unroll
-            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(s[c][i]));
+            for (int i = 0; i < 16; ++i)
+              mx8[i & 7] = fmax3(mx8[i & 7], __uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1]));
+          const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                 fmaxf(mx8[6], mx8[7]));
           const float m_new = mx * sl2;
           if (!have) {
             m_run = m_new;
@@ -416,31 +435,53 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (need) m_run = m_new;
             }
           }
-          float lsum = 0.f;
+          // x = s * scale*log2(e) - m and the row sum in packed fp32x2 arithmetic.
+          // Each half of P is published as soon as it is in TMEM.
+          const float2 sl2x2 = make_float2(sl2, sl2);
+          const float2 negm = make_float2(-m_run, -m_run);
+          float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
           for (int c = 0; c < NC; ++c) {
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float p0 = ex2_approx(fmaf(__uint_as_float(s[c][2 * i]), sl2, -m_run));
-              const float p1 = ex2_approx(fmaf(__uint_as_float(s[c][2 * i + 1]), sl2, -m_run));
-              lsum += p0 + p1;
+              const float2 xv = __ffma2_rn(
+                  make_float2(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])), sl2x2, negm);
+              float p0, p1;
+              if (kPolyEvery > 0 && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
+                const float2 pv = exp2_poly3x2(xv);
+                p0 = pv.x;
+                p1 = pv.y;
+              } else {
+                p0 = ex2_approx(xv.x);
+                p1 = ex2_approx(xv.y);
+              }
+              ls[i & 1] = __fadd2_rn(ls[i & 1], make_float2(p0, p1));
               pk[i] = pack_bf16x2(p0, p1);
             }
             tmem_st16(tS + c * 16, pk);
+            if (c == NC / 2 - 1 || c == NC - 1) {
+              tmem_wait_st();
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&sm.p_full[X][c == NC - 1 ? 1 : 0]);
+            }
           }
-          l_run += lsum;
+          l_run += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
         } else {
           uint32_t z[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) z[i] = 0u;
 #pragma unroll
           for (int c = 0; c < NC; ++c) tmem_st16(tS + c * 16, z);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&sm.p_full[X][0]);
+            mbar_arrive(&sm.p_full[X][1]);
+          }
         }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.p_full[X]);
       }
       if (!ok) break;
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_full[X], on & 1, abort_flag, P.status))) break;
