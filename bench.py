@@ -42,6 +42,30 @@ import synthetic as S  # noqa: E402
 METRIC = "sparse attn ms/call & effective TFLOP/s (Wan-14B 720p shape) vs own dense"
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
+# launch from a one-pass ncu capture, per workload, with the sha256 prefix of
+# the kernel source they were taken on. They are reported only while the source
+# is unchanged; after any change the traffic is unknown and reported as null.
+ATTN_TRAFFIC = {
+    "wan14b-720p": {"bytes": 2.54e9 + 764.24e6, "src": "d8063faaf0ab5a25"},
+    "wan14b-480p": {"bytes": 1.023992e9 + 321.768704e6, "src": "d8063faaf0ab5a25"},
+}
+ATTN_SRC = os.path.join(ROOT, "block_sparse_attention_video_b200", "csrc", "attn_sm100.cu")
+
+
+def _attn_traffic(workload: str):
+    import hashlib
+    rec = ATTN_TRAFFIC.get(workload)
+    if rec is None:
+        return None
+    try:
+        with open(ATTN_SRC, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    return rec["bytes"] if sha.startswith(rec["src"]) else None
+
+
 def _peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -234,7 +258,7 @@ def run_fvattn(args):
     attn_ms = [a.elapsed_time(b) for a, b in ev]
     ms_attn = sum(attn_ms) / len(attn_ms)
     ms_step_max = _max_over_ranks(dist, ms_step)
-    launches_per_step = 7   # gather_pool, route_select, permute V, plan x2, attention, inverse permute
+    launches_per_step = 8   # gather_pool, route_select, permute V, plan x3, attention, inverse permute
 
     # ---- the build's own dense kernel at the same shape
     dense_ms = []
@@ -297,7 +321,8 @@ def run_fvattn(args):
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "grid": list(w.grid),
                    "tiles": list(w.tile), "block": w.block, "p": w.p, "k_min": w.k_min,
-                   "l2": "inputs larger than L2 (Q, K, V 774 MB each); no flush",
+                   "l2": f"inputs larger than L2 (Q, K, V {w.B * w.H * w.N * w.d * 2 / 1e6:.0f} MB each); "
+                         f"no flush",
                    "parallelism": f"independent replicas x{world}"},
         "ms_per_call": ms_step_max,
         "attention_ms_per_launch": ms_attn,
@@ -310,7 +335,9 @@ def run_fvattn(args):
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_sm100_kernel", "achieved": achieved,
                      "peak": pk["bf16_sus"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_sus"],
                      "peak_kind": f"{pk['source']} bf16 sustained (kernel timed inside a long step)",
-                     "frac_of_burst_peak": achieved / pk["bf16"], "traffic": None},
+                     "frac_of_burst_peak": achieved / pk["bf16"],
+                     "traffic": _attn_traffic(w.name), "traffic_unit": "bytes per launch (DRAM read + write)",
+                     "algorithmic_bytes": 4 * w.B * w.H * path.nb * w.block * w.d * 2},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
