@@ -28,3 +28,10 @@ from .fvattn_oracle import (  # noqa: F401
     masked_attention_rows,
     dense_attention,
 )
+from .gsrs_oracle import (  # noqa: F401
+    block_lse_rows,
+    row_lse,
+    block_importance_row,
+    block_importance,
+    attention_recall,
+)
