@@ -208,6 +208,56 @@ def cpu_oracle_sample(w, q, k, v, kv_idx, kv_cnt, budget_s=15.0, seed=0):
     return flops / dt / 1e12, blocks, dt, cores
 
 
+def run_diag(F, w, path, stream, warmup):
+    dev = path.qp.device
+    nb, npad = path.nb, path.npad
+    lse = torch.empty((w.B, w.H, npad), dtype=torch.float32, device=dev)
+    blse = torch.empty((w.B, w.H, nb, npad), dtype=torch.float32, device=dev)
+    imp = torch.empty((w.B, w.H, nb, nb), dtype=torch.float32, device=dev)
+    rec = torch.empty((w.B, w.H, nb), dtype=torch.float32, device=dev)
+    wsd = F.alloc_workspace(F.fvattn_workspace_bytes(F.FVATTN_OP_DIAG, w.B, w.H, w.N, w.d, w.block), dev)
+
+    def timed(fn, reps):
+        for _ in range(max(1, warmup)):
+            fn()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    sparse_ms = timed(lambda: F.fvattn_sparse_fwd(path.qp, path.kp, path.vp, path.op, path.kv_idx,
+                                                  path.kv_cnt, w.N, w.block, path.ws_attn), 3)
+    sparse_blse_ms = timed(lambda: F.fvattn_sparse_fwd(path.qp, path.kp, path.vp, path.op, path.kv_idx,
+                                                       path.kv_cnt, w.N, w.block, path.ws_attn,
+                                                       lse=lse, block_lse=blse), 3)
+    imp_ms = timed(lambda: F.fvattn_block_importance(blse, lse, imp, w.N, w.block, wsd,
+                                                     kv_idx=path.kv_idx, kv_cnt=path.kv_cnt), 3)
+    sparse_sum = float(imp.sum(-1).sub(1).abs().max())
+    F.fvattn_dense_fwd(path.qp, path.kp, path.vp, path.op, w.N, w.block, path.ws_attn, lse=lse,
+                       block_lse=blse)
+    F.fvattn_block_importance(blse, lse, imp, w.N, w.block, wsd)
+    F.fvattn_attention_recall(imp, path.kv_idx, path.kv_cnt, rec, w.N, w.block, wsd)
+    torch.cuda.synchronize()
+    if F.fvattn_workspace_status(wsd) != F.FVATTN_OK or F.fvattn_workspace_status(path.ws_attn) != F.FVATTN_OK:
+        raise RuntimeError("kernel status word set in the diagnostic")
+    r = rec.float()
+    out = {"sparse_attention_ms": sparse_ms, "sparse_attention_with_block_lse_ms": sparse_blse_ms,
+           "block_lse_overhead": sparse_blse_ms / sparse_ms - 1.0, "importance_ms": imp_ms,
+           "sparse_importance_row_sum_max_err": sparse_sum,
+           "recall_of_routed_mask": {"mean": float(r.mean()), "p05": float(r.flatten().quantile(0.05)),
+                                     "min": float(r.min())},
+           "note": "GSRS block importance from block log-sum-exps; recall = dense importance captured by the "
+                   "routed lists"}
+    del blse, imp
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_fvattn(args):
     import block_sparse_attention_video_b200 as F
     dist, rank, world, local = _dist_setup(args.gpus)
@@ -272,6 +322,13 @@ def run_fvattn(args):
             dense_ms.append(a.elapsed_time(b))
     ms_dense = sum(dense_ms) / len(dense_ms)
     d_flops = dense_flops(w.B, w.H, w.N, w.d)
+
+    # ---- GSRS diagnostic (outside the timed region): cost of recording block
+    # log-sum-exps in the sparse launch, the importance kernel, and the attention
+    # recall of the routed mask under the dense attention's block importance.
+    diag = None
+    if not args.no_diag:
+        diag = run_diag(F, w, path, stream, args.warmup)
 
     # ---- e2e through the public API with pinned host buffers
     e2e = None
@@ -343,6 +400,8 @@ def run_fvattn(args):
     }
     if e2e is not None:
         line["e2e"] = e2e
+    if diag is not None:
+        line["diag"] = diag
     if not args.no_cpu_baseline:
         tf, nblk, secs, cores = cpu_oracle_sample(w, q, k, v, path.kv_idx, path.kv_cnt,
                                                   budget_s=args.cpu_budget)
@@ -417,6 +476,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="wan14b-720p", choices=sorted(S.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-diag", action="store_true", help="skip the GSRS block-importance diagnostic")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "fvattn":

@@ -8,6 +8,7 @@ fallback: importing it fails loudly if the library has not been built
 
 Entry points carry the C names: ``fvattn_permute``, ``fvattn_route``,
 ``fvattn_route_noalloc``, ``fvattn_sparse_fwd``, ``fvattn_dense_fwd``,
+``fvattn_block_importance``, ``fvattn_attention_recall``,
 ``fvattn_workspace_bytes``, ``fvattn_workspace_status``. ``FVAttnPath`` strings them into the full per-call
 path (route -> permute V -> block-sparse attention -> inverse permute) over
 buffers it allocates once with torch.
@@ -44,9 +45,11 @@ FVATTN_FP32 = 1
 FVATTN_OP_ROUTE = 0
 FVATTN_OP_SPARSE_FWD = 1
 FVATTN_OP_DENSE_FWD = 2
+FVATTN_OP_DIAG = 3
 
 EXPORTED = ("fvattn_workspace_bytes", "fvattn_permute", "fvattn_route", "fvattn_route_noalloc",
-            "fvattn_sparse_fwd", "fvattn_dense_fwd", "fvattn_workspace_status", "fvattn_status_string")
+            "fvattn_sparse_fwd", "fvattn_dense_fwd", "fvattn_block_importance", "fvattn_attention_recall",
+            "fvattn_workspace_status", "fvattn_status_string")
 
 
 class Grid(ctypes.Structure):
@@ -83,13 +86,19 @@ _lib.fvattn_route_noalloc.argtypes = [_c_void_p, _c_void_p, _c_int, _c_int, _c_i
                                       _c_void_p, _c_void_p, _c_void_p, _c_void_p]
 _lib.fvattn_route_noalloc.restype = _c_int
 _lib.fvattn_sparse_fwd.argtypes = [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
-                                   _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
-                                   _c_int, _c_float, _c_void_p, _c_size_t, _c_void_p]
+                                   _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int,
+                                   _c_int, _c_int, _c_float, _c_void_p, _c_size_t, _c_void_p]
 _lib.fvattn_sparse_fwd.restype = _c_int
-_lib.fvattn_dense_fwd.argtypes = [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+_lib.fvattn_dense_fwd.argtypes = [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                                   _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
                                   _c_void_p, _c_size_t, _c_void_p]
 _lib.fvattn_dense_fwd.restype = _c_int
+_lib.fvattn_block_importance.argtypes = [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int,
+                                         _c_int, _c_int, _c_void_p, _c_void_p, _c_size_t, _c_void_p]
+_lib.fvattn_block_importance.restype = _c_int
+_lib.fvattn_attention_recall.argtypes = [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int,
+                                         _c_int, _c_void_p, _c_void_p, _c_size_t, _c_void_p]
+_lib.fvattn_attention_recall.restype = _c_int
 _lib.fvattn_workspace_status.argtypes = [_c_void_p, _c_void_p]
 _lib.fvattn_workspace_status.restype = _c_int
 _lib.fvattn_status_string.argtypes = [_c_int]
@@ -175,29 +184,56 @@ def fvattn_route_noalloc(q, k, grid: Grid, p: float, k_min: int, kv_idx, kv_cnt,
 
 
 def fvattn_sparse_fwd(qp, kp, vp, out, kv_idx, kv_cnt, N: int, block: int, workspace,
-                      scale=None, lse=None, stream=None):
-    """Block-sparse attention over permuted [B,H,Npad,d] tensors."""
-    _need_cuda(qp, kp, vp, out, kv_idx, kv_cnt, workspace, lse)
+                      scale=None, lse=None, block_lse=None, stream=None):
+    """Block-sparse attention over permuted [B,H,Npad,d] tensors; optional lse
+    [B,H,Npad] and block_lse [B,H,nb,Npad] (fp32) outputs."""
+    _need_cuda(qp, kp, vp, out, kv_idx, kv_cnt, workspace, lse, block_lse)
     B, H, _, d = qp.shape
     sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    _check(_lib.fvattn_sparse_fwd(_ptr(qp), _ptr(kp), _ptr(vp), _ptr(out), _ptr(lse), _ptr(kv_idx),
-                                  _ptr(kv_cnt), B, H, N, d, _dtype_code(qp), block, sc,
+    _check(_lib.fvattn_sparse_fwd(_ptr(qp), _ptr(kp), _ptr(vp), _ptr(out), _ptr(lse), _ptr(block_lse),
+                                  _ptr(kv_idx), _ptr(kv_cnt), B, H, N, d, _dtype_code(qp), block, sc,
                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
                                   _stream(stream)), "fvattn_sparse_fwd")
     return out
 
 
 def fvattn_dense_fwd(qp, kp, vp, out, N: int, block: int, workspace, scale=None, lse=None,
-                     stream=None):
+                     block_lse=None, stream=None):
     """Dense attention over permuted [B,H,Npad,d] tensors (every key block)."""
-    _need_cuda(qp, kp, vp, out, workspace, lse)
+    _need_cuda(qp, kp, vp, out, workspace, lse, block_lse)
     B, H, _, d = qp.shape
     sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    _check(_lib.fvattn_dense_fwd(_ptr(qp), _ptr(kp), _ptr(vp), _ptr(out), _ptr(lse), B, H, N, d,
+    _check(_lib.fvattn_dense_fwd(_ptr(qp), _ptr(kp), _ptr(vp), _ptr(out), _ptr(lse), _ptr(block_lse),
+                                 B, H, N, d,
                                  _dtype_code(qp), block, sc, _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream)),
            "fvattn_dense_fwd")
     return out
+
+
+def fvattn_block_importance(block_lse, lse, importance, N: int, block: int, workspace,
+                            kv_idx=None, kv_cnt=None, stream=None):
+    """Exact block importance [B,H,nb,nb] from an attention call's block_lse and lse
+    (kv_idx/kv_cnt: the call's lists; None for a dense call)."""
+    _need_cuda(block_lse, lse, importance, workspace, kv_idx, kv_cnt)
+    B, H = lse.shape[:2]
+    _check(_lib.fvattn_block_importance(_ptr(block_lse), _ptr(lse), _ptr(kv_idx), _ptr(kv_cnt), B, H,
+                                        N, block, _ptr(importance), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _stream(stream)),
+           "fvattn_block_importance")
+    return importance
+
+
+def fvattn_attention_recall(importance, kv_idx, kv_cnt, recall, N: int, block: int, workspace,
+                            stream=None):
+    """Per query block, the dense importance captured by the lists: recall [B,H,nb]."""
+    _need_cuda(importance, kv_idx, kv_cnt, recall, workspace)
+    B, H = kv_cnt.shape[:2]
+    _check(_lib.fvattn_attention_recall(_ptr(importance), _ptr(kv_idx), _ptr(kv_cnt), B, H, N, block,
+                                        _ptr(recall), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _stream(stream)),
+           "fvattn_attention_recall")
+    return recall
 
 
 def fvattn_workspace_status(workspace, stream=None) -> int:

@@ -18,14 +18,20 @@ cudaError_t launch_route_select(const float* qbar, const float* kbar, int BH, in
                                 float scale, float p, int k_min, int* kv_idx, int* kv_cnt,
                                 unsigned long long* head_work, int* status, cudaStream_t st);
 cudaError_t launch_attn_simt(const void* q, const void* k, const void* v, void* o, float* lse,
-                             const int* kv_idx, const int* kv_cnt, int BH, int N, int d, int bs,
-                             bool bf16, float scale, int* status, cudaStream_t st);
+                             float* blse, const int* kv_idx, const int* kv_cnt, int BH, int N,
+                             int d, int bs, bool bf16, float scale, int* status, cudaStream_t st);
 cudaError_t launch_attn_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                              void* out, float* lse, const int* kv_idx, const int* kv_cnt,
+                              void* out, float* lse, float* blse, const int* kv_idx,
+                              const int* kv_cnt,
                               uint32_t* ulist, int* ucnt, int* local_order,
                               unsigned long long* head_total, int* head_order, int BH, int N,
                               int nb, int bs, float scale, int* status,
                               unsigned long long* counter, int num_sms, cudaStream_t st);
+cudaError_t launch_block_importance(const float* blse, const float* lse, const int* kv_idx,
+                                    const int* kv_cnt, int BH, int N, int bs, float* importance,
+                                    int* status, cudaStream_t st);
+cudaError_t launch_attention_recall(const float* importance, const int* kv_idx, const int* kv_cnt,
+                                    int BH, int nb, float* recall, int* status, cudaStream_t st);
 }  // namespace fvattn
 
 namespace {
@@ -149,13 +155,14 @@ fvattn_status check_ws(const void* ws, size_t have, size_t need) {
 
 // Common validation and dispatch of the attention forward (sparse or dense).
 fvattn_status attention_fwd(const void* qp, const void* kp, const void* vp, void* op, float* lse,
-                            const int32_t* kv_idx, const int32_t* kv_cnt, bool sparse, int B,
+                            float* block_lse, const int32_t* kv_idx, const int32_t* kv_cnt, bool sparse, int B,
                             int H, int N, int d, fvattn_dtype dtype, int block, float scale,
                             void* ws, size_t ws_bytes, void* stream) {
   if (!qp || !kp || !vp || !op) return FVATTN_ERR_INVALID_ARG;
   if (!aligned(qp, 16) || !aligned(kp, 16) || !aligned(vp, 16) || !aligned(op, 16))
     return FVATTN_ERR_INVALID_ARG;
   if (lse && !aligned(lse, 4)) return FVATTN_ERR_INVALID_ARG;
+  if (block_lse && !aligned(block_lse, 4)) return FVATTN_ERR_INVALID_ARG;
   if (sparse && (!kv_idx || !kv_cnt || !aligned(kv_idx, 4) || !aligned(kv_cnt, 4)))
     return FVATTN_ERR_INVALID_ARG;
   if (!valid_dtype(dtype) || !valid_sizes(B, H, N, d, block)) return FVATTN_ERR_INVALID_ARG;
@@ -174,7 +181,7 @@ fvattn_status attention_fwd(const void* qp, const void* kp, const void* vp, void
 
   const bool tensor_core = dtype == FVATTN_BF16 && d == 128;
   if (!tensor_core) {
-    return from_cuda(fvattn::launch_attn_simt(qp, kp, vp, op, lse, sparse ? kv_idx : nullptr,
+    return from_cuda(fvattn::launch_attn_simt(qp, kp, vp, op, lse, block_lse, sparse ? kv_idx : nullptr,
                                               sparse ? kv_cnt : nullptr, BH, N, d, block,
                                               dtype == FVATTN_BF16, scale, &hdr->status, st));
   }
@@ -199,7 +206,7 @@ fvattn_status attention_fwd(const void* qp, const void* kp, const void* vp, void
     head_order = reinterpret_cast<int*>(base + w.head_order);
   }
   return from_cuda(fvattn::launch_attn_sm100(
-      tq, tk, tv, op, lse, sparse ? kv_idx : nullptr, sparse ? kv_cnt : nullptr, ulist, ucnt,
+      tq, tk, tv, op, lse, block_lse, sparse ? kv_idx : nullptr, sparse ? kv_cnt : nullptr, ulist, ucnt,
       local_order, head_total, head_order, BH, N, nb, block, scale, &hdr->status, &hdr->counter,
       sms, st));
 }
@@ -214,6 +221,7 @@ size_t fvattn_workspace_bytes(fvattn_op op, int B, int H, int N, int d, int bloc
     case FVATTN_OP_ROUTE: return route_ws(B, H, N, d, block).total;
     case FVATTN_OP_SPARSE_FWD: return sparse_ws(B, H, N, block).total;
     case FVATTN_OP_DENSE_FWD: return kWsHeaderBytes;
+    case FVATTN_OP_DIAG: return kWsHeaderBytes;
   }
   return 0;
 }
@@ -275,19 +283,56 @@ fvattn_status fvattn_route(const void* q, const void* k, int B, int H, int N, in
 }
 
 fvattn_status fvattn_sparse_fwd(const void* qp, const void* kp, const void* vp, void* op,
-                                float* lse, const int32_t* kv_idx, const int32_t* kv_cnt, int B,
-                                int H, int N, int d, fvattn_dtype dtype, int block, float scale,
-                                void* workspace, size_t workspace_bytes, void* stream) {
-  return attention_fwd(qp, kp, vp, op, lse, kv_idx, kv_cnt, true, B, H, N, d, dtype, block,
-                       scale, workspace, workspace_bytes, stream);
+                                float* lse, float* block_lse, const int32_t* kv_idx,
+                                const int32_t* kv_cnt, int B, int H, int N, int d,
+                                fvattn_dtype dtype, int block, float scale, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  return attention_fwd(qp, kp, vp, op, lse, block_lse, kv_idx, kv_cnt, true, B, H, N, d, dtype,
+                       block, scale, workspace, workspace_bytes, stream);
 }
 
 fvattn_status fvattn_dense_fwd(const void* qp, const void* kp, const void* vp, void* op,
-                               float* lse, int B, int H, int N, int d, fvattn_dtype dtype,
-                               int block, float scale, void* workspace, size_t workspace_bytes,
-                               void* stream) {
-  return attention_fwd(qp, kp, vp, op, lse, nullptr, nullptr, false, B, H, N, d, dtype, block,
-                       scale, workspace, workspace_bytes, stream);
+                               float* lse, float* block_lse, int B, int H, int N, int d,
+                               fvattn_dtype dtype, int block, float scale, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  return attention_fwd(qp, kp, vp, op, lse, block_lse, nullptr, nullptr, false, B, H, N, d,
+                       dtype, block, scale, workspace, workspace_bytes, stream);
+}
+
+fvattn_status fvattn_block_importance(const float* block_lse, const float* lse,
+                                      const int32_t* kv_idx, const int32_t* kv_cnt, int B, int H,
+                                      int N, int block, float* importance, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  if (!block_lse || !lse || !importance) return FVATTN_ERR_INVALID_ARG;
+  if ((kv_idx == nullptr) != (kv_cnt == nullptr)) return FVATTN_ERR_INVALID_ARG;
+  if (!aligned(block_lse, 4) || !aligned(lse, 4) || !aligned(importance, 4) ||
+      (kv_idx && (!aligned(kv_idx, 4) || !aligned(kv_cnt, 4))))
+    return FVATTN_ERR_INVALID_ARG;
+  if (!valid_sizes(B, H, N, 64, block)) return FVATTN_ERR_INVALID_ARG;
+  const fvattn_status wst = check_ws(workspace, workspace_bytes, kWsHeaderBytes);
+  if (wst != FVATTN_OK) return wst;
+  auto st = static_cast<cudaStream_t>(stream);
+  auto hdr = static_cast<fvattn::WsHeader*>(workspace);
+  if (cudaMemsetAsync(workspace, 0, kWsHeaderBytes, st) != cudaSuccess) return FVATTN_ERR_CUDA;
+  return from_cuda(fvattn::launch_block_importance(block_lse, lse, kv_idx, kv_cnt, B * H, N, block,
+                                                   importance, &hdr->status, st));
+}
+
+fvattn_status fvattn_attention_recall(const float* importance, const int32_t* kv_idx,
+                                      const int32_t* kv_cnt, int B, int H, int N, int block,
+                                      float* recall, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+  if (!importance || !kv_idx || !kv_cnt || !recall) return FVATTN_ERR_INVALID_ARG;
+  if (!aligned(importance, 4) || !aligned(kv_idx, 4) || !aligned(kv_cnt, 4) || !aligned(recall, 4))
+    return FVATTN_ERR_INVALID_ARG;
+  if (!valid_sizes(B, H, N, 64, block)) return FVATTN_ERR_INVALID_ARG;
+  const fvattn_status wst = check_ws(workspace, workspace_bytes, kWsHeaderBytes);
+  if (wst != FVATTN_OK) return wst;
+  auto st = static_cast<cudaStream_t>(stream);
+  auto hdr = static_cast<fvattn::WsHeader*>(workspace);
+  if (cudaMemsetAsync(workspace, 0, kWsHeaderBytes, st) != cudaSuccess) return FVATTN_ERR_CUDA;
+  return from_cuda(fvattn::launch_attention_recall(importance, kv_idx, kv_cnt, B * H,
+                                                   num_blocks(N, block), recall, &hdr->status, st));
 }
 
 fvattn_status fvattn_workspace_status(const void* workspace, void* stream) {

@@ -8,6 +8,9 @@
 // a running max m, a running sum l and 32 output accumulators, and updates them
 // exactly for every valid key of every selected block:
 //   m' = max(m, s),  l' = l*exp(m-m') + exp(s-m'),  o' = o*exp(m-m') + exp(s-m')*v.
+// When block_lse is requested, the CTAs of the first output slice also keep a
+// per-block max and sum and store each selected block's log-sum-exp
+// [GSRS §5.3: per-block statistics recorded during the attention pass].
 #include "common.cuh"
 
 namespace fvattn {
@@ -34,7 +37,8 @@ __device__ __forceinline__ __nv_bfloat16 store_cast<__nv_bfloat16>(float v) {
 template <typename T, int D, int BS>
 __global__ void __launch_bounds__(BS)
     attn_simt_kernel(const T* __restrict__ qp, const T* __restrict__ kp, const T* __restrict__ vp,
-                     T* __restrict__ op, float* __restrict__ lse, const int* __restrict__ kv_idx,
+                     T* __restrict__ op, float* __restrict__ lse, float* __restrict__ blse,
+                     const int* __restrict__ kv_idx,
                      const int* __restrict__ kv_cnt, int nb, int N, float scale, int* status) {
   extern __shared__ float4 smem_f4[];
   float* Qs = reinterpret_cast<float*>(smem_f4);   // BS x (D+1)
@@ -63,6 +67,7 @@ __global__ void __launch_bounds__(BS)
     list = kv_idx + (static_cast<size_t>(bh) * nb + i) * nb;
   }
 
+  const bool want_blse = blse != nullptr && blockIdx.y == 0;
   float m = -INFINITY, l = 0.f;
   float acc[kSlice];
 #pragma unroll
@@ -85,11 +90,20 @@ __global__ void __launch_bounds__(BS)
       Vs[r * (kSlice + 1) + c] = load_elem<T>(vp + (head + static_cast<size_t>(j) * BS + r) * D + d0 + c);
     }
     __syncthreads();
+    float bm = -INFINITY, bl = 0.f;
     for (int c = 0; c < valid; ++c) {
       float s = 0.f;
 #pragma unroll 8
       for (int kk = 0; kk < D; ++kk) s = fmaf(Qs[row * (D + 1) + kk], Ks[c * (D + 1) + kk], s);
       s *= scale;
+      if (want_blse) {
+        if (s > bm) {
+          bl = bl * expf(bm - s) + 1.f;
+          bm = s;
+        } else {
+          bl += expf(s - bm);
+        }
+      }
       if (s > m) {
         const float corr = expf(m - s);
         l = l * corr + 1.f;
@@ -103,6 +117,7 @@ __global__ void __launch_bounds__(BS)
         for (int e = 0; e < kSlice; ++e) acc[e] = fmaf(w, Vs[c * (kSlice + 1) + e], acc[e]);
       }
     }
+    if (want_blse) blse[(static_cast<size_t>(bh) * nb + j) * npad + static_cast<size_t>(i) * BS + row] = bm + logf(bl);
   }
   const float inv = 1.f / l;
   T* orow = op + (head + static_cast<size_t>(i) * BS + row) * D + d0;
@@ -113,7 +128,7 @@ __global__ void __launch_bounds__(BS)
 
 template <typename T, int D, int BS>
 static cudaError_t launch_simt_t(const void* q, const void* k, const void* v, void* o, float* lse,
-                                 const int* kv_idx, const int* kv_cnt, int BH, int nb, int N,
+                                 float* blse, const int* kv_idx, const int* kv_cnt, int BH, int nb, int N,
                                  float scale, int* status, cudaStream_t st) {
   const size_t smem = (static_cast<size_t>(BS) * (D + 1) * 2 + static_cast<size_t>(BS) * (kSlice + 1)) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(attn_simt_kernel<T, D, BS>,
@@ -122,17 +137,17 @@ static cudaError_t launch_simt_t(const void* q, const void* k, const void* v, vo
   const dim3 grid(static_cast<unsigned>(BH) * nb, D / kSlice);
   attn_simt_kernel<T, D, BS><<<grid, BS, smem, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), static_cast<T*>(o),
-      lse, kv_idx, kv_cnt, nb, N, scale, status);
+      lse, blse, kv_idx, kv_cnt, nb, N, scale, status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_attn_simt(const void* q, const void* k, const void* v, void* o, float* lse,
-                             const int* kv_idx, const int* kv_cnt, int BH, int N, int d, int bs,
+                             float* blse, const int* kv_idx, const int* kv_cnt, int BH, int N, int d, int bs,
                              bool bf16, float scale, int* status, cudaStream_t st) {
   const int nb = (N + bs - 1) / bs;
 #define FVATTN_SIMT_CASE(T, D_, BS_)                                                         \
   if (d == D_ && bs == BS_)                                                                  \
-    return launch_simt_t<T, D_, BS_>(q, k, v, o, lse, kv_idx, kv_cnt, BH, nb, N, scale, status, st);
+    return launch_simt_t<T, D_, BS_>(q, k, v, o, lse, blse, kv_idx, kv_cnt, BH, nb, N, scale, status, st);
   if (bf16) {
     FVATTN_SIMT_CASE(__nv_bfloat16, 64, 64)
     FVATTN_SIMT_CASE(__nv_bfloat16, 64, 128)

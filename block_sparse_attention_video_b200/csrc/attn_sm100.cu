@@ -94,6 +94,7 @@ struct Params {
   const int* local_order;   // [B*H*ngroups] (bh, rank) -> group
   __nv_bfloat16* out;
   float* lse;
+  float* blse;              // nullable [B*H, nb, npad]: per (key block, row) log-sum-exp
   int* status;
   unsigned long long* counter;
 };
@@ -467,7 +468,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (lane == 0) mbar_arrive(&sm.p_full[X][c == NC - 1 ? 1 : 0]);
             }
           }
-          l_run += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
+          const float l_blk = (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
+          l_run += l_blk;
+          // Block log-sum-exp of this row over this key block [GSRS §5.3]: the
+          // exponentials above are relative to m_run, so it is m_run + log2 of
+          // their sum, converted to the natural base.
+          if (P.blse) {
+            const int qrow = x.grp * kUnitRows + X * 128 + row;
+            if (qrow < P.npad)
+              P.blse[(static_cast<size_t>(x.bh) * P.nb + (e & 0xFFFFu)) * P.npad + qrow] =
+                  (m_run + __log2f(l_blk)) * kLn2;
+          }
         } else {
           uint32_t z[16];
 #pragma unroll
@@ -671,7 +682,8 @@ static cudaError_t launch_bn(const CUtensorMap& tq, const CUtensorMap& tk, const
 }
 
 cudaError_t launch_attn_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                              void* out, float* lse, const int* kv_idx, const int* kv_cnt,
+                              void* out, float* lse, float* blse, const int* kv_idx,
+                              const int* kv_cnt,
                               uint32_t* ulist, int* ucnt, int* local_order,
                               unsigned long long* head_total, int* head_order, int BH, int N,
                               int nb, int bs, float scale, int* status,
@@ -702,6 +714,7 @@ cudaError_t launch_attn_sm100(const CUtensorMap& tq, const CUtensorMap& tk, cons
   P.local_order = local_order;
   P.out = static_cast<__nv_bfloat16*>(out);
   P.lse = lse;
+  P.blse = blse;
   P.status = status;
   P.counter = counter;
   return bs == 64 ? launch_bn<64>(tq, tk, tv, P, num_sms, st) : launch_bn<128>(tq, tk, tv, P, num_sms, st);

@@ -20,6 +20,9 @@
  *                                                        [FVAttn §2.1; GSRS §3.2, §A.1]
  *   fvattn_dense_fwd  the same kernel with every block selected (the dense
  *                     baseline every page compares against)
+ * Diagnostic of mask quality, from statistics the attention kernels record:
+ *   fvattn_block_importance  exact block importance   [GSRS §5.3, §A.2, §A.3]
+ *   fvattn_attention_recall  attention recall of a mask            [GSRS §3.2]
  *
  * Conventions (every entry point):
  *   - Tensors are dense, row-major, on the current CUDA device. A token row of
@@ -82,7 +85,8 @@ typedef struct {
 typedef enum {
   FVATTN_OP_ROUTE = 0,
   FVATTN_OP_SPARSE_FWD = 1,
-  FVATTN_OP_DENSE_FWD = 2
+  FVATTN_OP_DENSE_FWD = 2,
+  FVATTN_OP_DIAG = 3      /* fvattn_block_importance, fvattn_attention_recall */
 } fvattn_op;
 
 /* Workspace bytes needed by `op` for these sizes (0 if the sizes are invalid).
@@ -150,7 +154,13 @@ FVATTN_API fvattn_status fvattn_route_noalloc(const void* q, const void* k, int 
  * < N) of the key blocks kv_idx[b,h,i,0..cnt) of scale * q.k, times V.
  * lse: optional [B,H,Npad] fp32 natural-log sum of exp of the scaled logits
  * over the attended keys (NULL to skip). Rows >= N of op and lse are written
- * but carry no meaning. kv_idx/kv_cnt as produced by fvattn_route (any order
+ * but carry no meaning.
+ * block_lse: optional [B,H,nb,Npad] fp32 (key block major) [GSRS §5.3, §A.3]:
+ * entry (b,h,j,r) = natural-log sum of exp of the scaled logits of row r over
+ * the valid keys of key block j, written only for the (row, key block) pairs
+ * the row attends (its block's list); other entries are left untouched. With
+ * lse it gives the exact block importance (fvattn_block_importance). NULL to
+ * skip; the tensor-core kernel then does no extra work. kv_idx/kv_cnt as produced by fvattn_route (any order
  * of entries within a row is accepted). scale > 0 (1/sqrt(d) is the usual).
  * BF16 with d == 128 (block 64 or 128) runs the tcgen05/TMEM tensor-core
  * kernel (bf16 MMA, fp32 accumulation and softmax, P rounded to bf16); it
@@ -159,19 +169,48 @@ FVATTN_API fvattn_status fvattn_route_noalloc(const void* q, const void* k, int 
  * kernel (fp32 throughout).
  * Workspace: fvattn_workspace_bytes(FVATTN_OP_SPARSE_FWD, ...). */
 FVATTN_API fvattn_status fvattn_sparse_fwd(const void* qp, const void* kp, const void* vp,
-                                void* op, float* lse, const int32_t* kv_idx,
+                                void* op, float* lse, float* block_lse,
+                                const int32_t* kv_idx,
                                 const int32_t* kv_cnt, int B, int H, int N, int d,
                                 fvattn_dtype dtype, int block, float scale,
                                 void* workspace, size_t workspace_bytes,
                                 void* stream);
 
-/* Dense attention forward: fvattn_sparse_fwd with every key block selected.
+/* Dense attention forward: fvattn_sparse_fwd with every key block selected
+ * (block_lse, when given, is written for every (row, key block) pair).
  * Workspace: fvattn_workspace_bytes(FVATTN_OP_DENSE_FWD, ...). */
 FVATTN_API fvattn_status fvattn_dense_fwd(const void* qp, const void* kp, const void* vp,
-                               void* op, float* lse, int B, int H, int N, int d,
+                               void* op, float* lse, float* block_lse, int B, int H, int N,
+                               int d,
                                fvattn_dtype dtype, int block, float scale,
                                void* workspace, size_t workspace_bytes,
                                void* stream);
+
+/* Exact block importance [GSRS §5.3, §A.2, §A.3] from the block_lse and lse
+ * of one attention call (sparse or dense, same B, H, N, block):
+ *   importance[b,h,i,j] = (1/n_i) * sum over the valid rows r of query block i
+ *                         of exp(block_lse[b,h,j,r] - lse[b,h,r])
+ * for the key blocks j in row (b,h,i) of kv_idx/kv_cnt (the evaluated set;
+ * both NULL = every block, for a dense call), and 0 for every other j;
+ * n_i = valid rows of block i. Each row of importance sums to 1 over its
+ * evaluated set. importance [B,H,nb,nb] fp32 is fully written.
+ * Workspace: fvattn_workspace_bytes(FVATTN_OP_DIAG, ...) (status word only). */
+FVATTN_API fvattn_status fvattn_block_importance(const float* block_lse, const float* lse,
+                                                 const int32_t* kv_idx, const int32_t* kv_cnt,
+                                                 int B, int H, int N, int block,
+                                                 float* importance, void* workspace,
+                                                 size_t workspace_bytes, void* stream);
+
+/* Attention recall of a block mask [GSRS §3.2]: the fraction of the attention
+ * weight that the listed blocks capture,
+ *   recall[b,h,i] = sum over t < kv_cnt[b,h,i] of importance[b,h,i,kv_idx[b,h,i,t]],
+ * where importance comes from fvattn_block_importance of a dense call (so it
+ * is normalised over every key). recall [B,H,nb] fp32.
+ * Workspace: fvattn_workspace_bytes(FVATTN_OP_DIAG, ...). */
+FVATTN_API fvattn_status fvattn_attention_recall(const float* importance, const int32_t* kv_idx,
+                                                 const int32_t* kv_cnt, int B, int H, int N,
+                                                 int block, float* recall, void* workspace,
+                                                 size_t workspace_bytes, void* stream);
 
 /* Synchronizes `stream` and returns the status word that the kernels of the
  * last call using `workspace` recorded (FVATTN_OK if none). */

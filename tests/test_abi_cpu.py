@@ -24,6 +24,7 @@ def _declared_symbols():
 def test_header_declares_the_four_calls_and_helpers():
     decl = _declared_symbols()
     for name in ("fvattn_permute", "fvattn_route", "fvattn_sparse_fwd", "fvattn_dense_fwd",
+                 "fvattn_block_importance", "fvattn_attention_recall",
                  "fvattn_workspace_bytes", "fvattn_workspace_status", "fvattn_status_string"):
         assert name in decl
 
@@ -106,8 +107,8 @@ def test_route_rejects(kw, status):
 
 
 def _sparse(qp=FAKE, op=FAKE, idx=FAKE, scale=0.125, ws=FAKE, ws_bytes=1 << 30, B=1, H=2, N=256,
-            d=64, block=64, dt=F.FVATTN_FP32):
-    return F._lib.fvattn_sparse_fwd(qp, FAKE, FAKE, op, None, idx, FAKE, B, H, N, d, dt, block,
+            d=64, block=64, dt=F.FVATTN_FP32, blse=None):
+    return F._lib.fvattn_sparse_fwd(qp, FAKE, FAKE, op, None, blse, idx, FAKE, B, H, N, d, dt, block,
                                     scale, ws, ws_bytes, None)
 
 
@@ -123,13 +124,56 @@ def _sparse(qp=FAKE, op=FAKE, idx=FAKE, scale=0.125, ws=FAKE, ws_bytes=1 << 30, 
     (dict(B=100, H=100), F.FVATTN_ERR_INVALID_ARG),        # B*H above the planner's limit
     (dict(ws_bytes=16), F.FVATTN_ERR_WORKSPACE),
     (dict(ws=None), F.FVATTN_ERR_WORKSPACE),
+    (dict(blse=FAKE + 2), F.FVATTN_ERR_INVALID_ARG),       # block_lse must be 4-byte aligned
 ])
 def test_sparse_rejects(kw, status):
     assert _sparse(**kw) == status
 
 
 def test_dense_rejects_and_status_rejects_bad_workspace():
-    assert F._lib.fvattn_dense_fwd(FAKE, FAKE, FAKE, None, None, 1, 1, 256, 64, F.FVATTN_FP32, 64,
-                                   0.125, FAKE, 1 << 20, None) == F.FVATTN_ERR_INVALID_ARG
+    assert F._lib.fvattn_dense_fwd(FAKE, FAKE, FAKE, None, None, None, 1, 1, 256, 64, F.FVATTN_FP32,
+                                   64, 0.125, FAKE, 1 << 20, None) == F.FVATTN_ERR_INVALID_ARG
     assert F._lib.fvattn_workspace_status(None, None) == F.FVATTN_ERR_WORKSPACE
     assert F._lib.fvattn_workspace_status(FAKE + 64, None) == F.FVATTN_ERR_WORKSPACE
+
+
+def _importance(blse=FAKE, lse=FAKE, idx=FAKE, cnt=FAKE, out=FAKE, B=1, H=2, N=256, block=64,
+                ws=FAKE, ws_bytes=256):
+    return F._lib.fvattn_block_importance(blse, lse, idx, cnt, B, H, N, block, out, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw, status", [
+    (dict(blse=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(lse=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(out=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(idx=None), F.FVATTN_ERR_INVALID_ARG),           # lists given half-way
+    (dict(cnt=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(lse=FAKE + 1), F.FVATTN_ERR_INVALID_ARG),
+    (dict(block=96), F.FVATTN_ERR_INVALID_ARG),
+    (dict(N=0), F.FVATTN_ERR_INVALID_ARG),
+    (dict(ws=None), F.FVATTN_ERR_WORKSPACE),
+    (dict(ws_bytes=64), F.FVATTN_ERR_WORKSPACE),
+])
+def test_block_importance_rejects(kw, status):
+    assert _importance(**kw) == status
+
+
+def _recall(imp=FAKE, idx=FAKE, cnt=FAKE, out=FAKE, B=1, H=2, N=256, block=64, ws=FAKE, ws_bytes=256):
+    return F._lib.fvattn_attention_recall(imp, idx, cnt, B, H, N, block, out, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw, status", [
+    (dict(imp=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(idx=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(cnt=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(out=FAKE + 2), F.FVATTN_ERR_INVALID_ARG),
+    (dict(B=0), F.FVATTN_ERR_INVALID_ARG),
+    (dict(ws=FAKE + 64), F.FVATTN_ERR_WORKSPACE),
+])
+def test_attention_recall_rejects(kw, status):
+    assert _recall(**kw) == status
+
+
+def test_diag_workspace_is_the_status_word():
+    assert F.fvattn_workspace_bytes(F.FVATTN_OP_DIAG, 1, 2, 256, 64, 64) == 256
+    assert F.fvattn_workspace_bytes(F.FVATTN_OP_DIAG, 1, 2, 256, 32, 64) == 0
