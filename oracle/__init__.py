@@ -11,6 +11,7 @@ Sources (page title, section):
            its English summary and its abstract page.
   [GSRS]   "Sparse Attention for Video Generation Acceleration via Growing
            Sparsity and Reduced Search".
+  [LVSA]   "LVSA: Training-Free Sparse Attention for Long Video Diffusion".
 """
 
 from .fvattn_oracle import (  # noqa: F401
@@ -34,4 +35,10 @@ from .gsrs_oracle import (  # noqa: F401
     block_importance_row,
     block_importance,
     attention_recall,
+)
+from .lvsa_oracle import (  # noqa: F401
+    global_frames,
+    attended_frames,
+    frame_mask,
+    lvsa_block_mask,
 )
