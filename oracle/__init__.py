@@ -42,3 +42,7 @@ from .lvsa_oracle import (  # noqa: F401
     frame_mask,
     lvsa_block_mask,
 )
+from .hilbert_oracle import (  # noqa: F401
+    hilbert_index,
+    hilbert_order,
+)
