@@ -208,7 +208,77 @@ def cpu_oracle_sample(w, q, k, v, kv_idx, kv_cnt, budget_s=15.0, seed=0):
     return flops / dt / 1e12, blocks, dt, cores
 
 
-def run_diag(F, w, path, stream, warmup):
+LVSA_WINDOW, LVSA_PERIOD, LVSA_STEP = 2, 8, 0
+
+
+def _median_ms(fn, stream, warmup, reps):
+    for _ in range(max(1, warmup)):
+        fn()
+    ts = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def run_lvsa(F, w, path, stream, warmup, eff_flops_fn):
+    """The LVSA static mask (window + rotating global frames) on the same tensors."""
+    dev = path.qp.device
+    idx = torch.empty_like(path.kv_idx)
+    cnt = torch.empty_like(path.kv_cnt)
+    hw = torch.empty_like(path.head_work)
+    ws = F.alloc_workspace(F.fvattn_workspace_bytes(F.FVATTN_OP_LVSA, w.B, w.H, w.N, w.d, w.block), dev)
+    gen_ms = _median_ms(lambda: F.fvattn_lvsa_lists(path.grid, LVSA_WINDOW, LVSA_PERIOD, LVSA_STEP, idx, cnt,
+                                                    hw, ws), stream, warmup, 3)
+    attn_ms = _median_ms(lambda: F.fvattn_sparse_fwd(path.qp, path.kp, path.vp, path.op, idx, cnt, w.N,
+                                                     w.block, path.ws_attn), stream, warmup, 3)
+    if F.fvattn_workspace_status(ws) != F.FVATTN_OK or F.fvattn_workspace_status(path.ws_attn) != F.FVATTN_OK:
+        raise RuntimeError("kernel status word set in the LVSA run")
+    idx_np, cnt_np = idx.cpu().numpy(), cnt.cpu().numpy()
+    eff = eff_flops_fn(idx_np, cnt_np, w.N, w.block, w.d)
+    hwn = hw.cpu().numpy().astype(np.float64)
+    return {"window": LVSA_WINDOW, "period": LVSA_PERIOD, "step": LVSA_STEP,
+            "density": float(cnt_np.mean() / path.nb), "lists_ms": gen_ms, "attention_ms": attn_ms,
+            "effective_tflops": eff / (attn_ms * 1e-3) / 1e12,
+            "head_work_max_over_mean": float(hwn.max() / hwn.mean()), "_lists": (idx, cnt)}
+
+
+def run_hilbert(F, w, q, k, v, stream, warmup, eff_flops_fn):
+    """The same call with blocks in Hilbert-curve order instead of 3-D tiles."""
+    dev = q.device
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    hpath = F.FVAttnPath(w.B, w.H, w.grid, w.tile, w.block, w.d, torch.bfloat16, w.p, w.k_min, device=dev,
+                         order="hilbert")
+    t1.record(stream)
+    torch.cuda.synchronize()
+    table_ms = t0.elapsed_time(t1)
+    hpath.route(q, k)
+    F.fvattn_permute(v, hpath.vp, hpath.grid)
+    attn_ms = _median_ms(lambda: hpath.attend(), stream, warmup, 3)
+    route_ms = _median_ms(lambda: hpath.route(q, k), stream, warmup, 3)
+    if F.fvattn_workspace_status(hpath.ws_route) != F.FVATTN_OK or \
+            F.fvattn_workspace_status(hpath.ws_attn) != F.FVATTN_OK:
+        raise RuntimeError("kernel status word set in the Hilbert-order run")
+    idx_np, cnt_np = hpath.kv_idx.cpu().numpy(), hpath.kv_cnt.cpu().numpy()
+    eff = eff_flops_fn(idx_np, cnt_np, w.N, w.block, w.d)
+    hwn = hpath.head_work.cpu().numpy().astype(np.float64)
+    diag = run_diag(F, w, hpath, stream, warmup)
+    out = {"table_build_ms": table_ms, "route_ms": route_ms, "density": float(cnt_np.mean() / hpath.nb),
+           "attention_ms": attn_ms, "effective_tflops": eff / (attn_ms * 1e-3) / 1e12,
+           "head_work_max_over_mean": float(hwn.max() / hwn.mean()),
+           "recall_of_routed_mask": diag["recall_of_routed_mask"]}
+    del hpath
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_diag(F, w, path, stream, warmup, lvsa_lists=None):
     dev = path.qp.device
     nb, npad = path.nb, path.npad
     lse = torch.empty((w.B, w.H, npad), dtype=torch.float32, device=dev)
@@ -242,6 +312,10 @@ def run_diag(F, w, path, stream, warmup):
                        block_lse=blse)
     F.fvattn_block_importance(blse, lse, imp, w.N, w.block, wsd)
     F.fvattn_attention_recall(imp, path.kv_idx, path.kv_cnt, rec, w.N, w.block, wsd)
+    rec_lvsa = None
+    if lvsa_lists is not None:
+        rec_lvsa = torch.empty_like(rec)
+        F.fvattn_attention_recall(imp, lvsa_lists[0], lvsa_lists[1], rec_lvsa, w.N, w.block, wsd)
     torch.cuda.synchronize()
     if F.fvattn_workspace_status(wsd) != F.FVATTN_OK or F.fvattn_workspace_status(path.ws_attn) != F.FVATTN_OK:
         raise RuntimeError("kernel status word set in the diagnostic")
@@ -253,6 +327,10 @@ def run_diag(F, w, path, stream, warmup):
                                      "min": float(r.min())},
            "note": "GSRS block importance from block log-sum-exps; recall = dense importance captured by the "
                    "routed lists"}
+    if rec_lvsa is not None:
+        rl = rec_lvsa.float()
+        out["recall_of_lvsa_mask"] = {"mean": float(rl.mean()), "p05": float(rl.flatten().quantile(0.05)),
+                                      "min": float(rl.min())}
     del blse, imp
     torch.cuda.empty_cache()
     return out
@@ -326,9 +404,16 @@ def run_fvattn(args):
     # ---- GSRS diagnostic (outside the timed region): cost of recording block
     # log-sum-exps in the sparse launch, the importance kernel, and the attention
     # recall of the routed mask under the dense attention's block importance.
+    hilbert = None
+    if not args.no_hilbert:
+        hilbert = run_hilbert(F, w, q, k, v, stream, args.warmup, eff_flops_fn=effective_flops)
+    lvsa = None
+    if not args.no_lvsa:
+        lvsa = run_lvsa(F, w, path, stream, args.warmup, eff_flops_fn=effective_flops)
     diag = None
     if not args.no_diag:
-        diag = run_diag(F, w, path, stream, args.warmup)
+        diag = run_diag(F, w, path, stream, args.warmup,
+                        lvsa_lists=(lvsa.pop("_lists") if lvsa is not None else None))
 
     # ---- e2e through the public API with pinned host buffers
     e2e = None
@@ -400,6 +485,11 @@ def run_fvattn(args):
     }
     if e2e is not None:
         line["e2e"] = e2e
+    if lvsa is not None:
+        lvsa.pop("_lists", None)
+        line["lvsa"] = lvsa
+    if hilbert is not None:
+        line["hilbert"] = hilbert
     if diag is not None:
         line["diag"] = diag
     if not args.no_cpu_baseline:
@@ -477,6 +567,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-diag", action="store_true", help="skip the GSRS block-importance diagnostic")
+    ap.add_argument("--no-lvsa", action="store_true", help="skip the LVSA static-mask measurement")
+    ap.add_argument("--no-hilbert", action="store_true", help="skip the Hilbert-order measurement")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "fvattn":

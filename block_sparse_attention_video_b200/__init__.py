@@ -8,7 +8,8 @@ fallback: importing it fails loudly if the library has not been built
 
 Entry points carry the C names: ``fvattn_permute``, ``fvattn_route``,
 ``fvattn_route_noalloc``, ``fvattn_sparse_fwd``, ``fvattn_dense_fwd``,
-``fvattn_block_importance``, ``fvattn_attention_recall``,
+``fvattn_block_importance``, ``fvattn_attention_recall``, ``fvattn_lvsa_lists``,
+``fvattn_hilbert_table``,
 ``fvattn_workspace_bytes``, ``fvattn_workspace_status``. ``FVAttnPath`` strings them into the full per-call
 path (route -> permute V -> block-sparse attention -> inverse permute) over
 buffers it allocates once with torch.
@@ -46,21 +47,32 @@ FVATTN_OP_ROUTE = 0
 FVATTN_OP_SPARSE_FWD = 1
 FVATTN_OP_DENSE_FWD = 2
 FVATTN_OP_DIAG = 3
+FVATTN_OP_LVSA = 4
+FVATTN_OP_HILBERT = 5
+
+FVATTN_ORDER_TILES = 0
+FVATTN_ORDER_TABLE = 1
 
 EXPORTED = ("fvattn_workspace_bytes", "fvattn_permute", "fvattn_route", "fvattn_route_noalloc",
             "fvattn_sparse_fwd", "fvattn_dense_fwd", "fvattn_block_importance", "fvattn_attention_recall",
+            "fvattn_lvsa_lists", "fvattn_hilbert_table",
             "fvattn_workspace_status", "fvattn_status_string")
 
 
 class Grid(ctypes.Structure):
-    """fvattn_grid: latent video grid (T, Hh, W), tiles (tt, th, tw), block size."""
+    """fvattn_grid: latent video grid (T, Hh, W), tiles (tt, th, tw), block size, and
+    block order (3-D tiles, or an explicit device table such as the Hilbert order)."""
     _fields_ = [("T", ctypes.c_int), ("Hh", ctypes.c_int), ("W", ctypes.c_int),
                 ("tt", ctypes.c_int), ("th", ctypes.c_int), ("tw", ctypes.c_int),
-                ("block", ctypes.c_int)]
+                ("block", ctypes.c_int), ("order", ctypes.c_int), ("table", ctypes.c_void_p)]
 
     @classmethod
-    def make(cls, grid, tile, block):
-        return cls(*grid, *tile, block)
+    def make(cls, grid, tile, block, table=None):
+        """Tile order, or the explicit order of ``table`` (an int32 CUDA tensor [N])."""
+        g = cls(*grid, *tile, block, FVATTN_ORDER_TILES if table is None else FVATTN_ORDER_TABLE,
+                None if table is None else table.data_ptr())
+        g._table = table          # keeps the table's storage alive with the grid
+        return g
 
     @property
     def N(self):
@@ -99,6 +111,11 @@ _lib.fvattn_block_importance.restype = _c_int
 _lib.fvattn_attention_recall.argtypes = [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int,
                                          _c_int, _c_void_p, _c_void_p, _c_size_t, _c_void_p]
 _lib.fvattn_attention_recall.restype = _c_int
+_lib.fvattn_lvsa_lists.argtypes = [_c_int, _c_int, ctypes.POINTER(Grid), _c_int, _c_int, _c_int, _c_void_p,
+                                   _c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_void_p]
+_lib.fvattn_lvsa_lists.restype = _c_int
+_lib.fvattn_hilbert_table.argtypes = [ctypes.POINTER(Grid), _c_void_p, _c_void_p, _c_size_t, _c_void_p]
+_lib.fvattn_hilbert_table.restype = _c_int
 _lib.fvattn_workspace_status.argtypes = [_c_void_p, _c_void_p]
 _lib.fvattn_workspace_status.restype = _c_int
 _lib.fvattn_status_string.argtypes = [_c_int]
@@ -236,6 +253,32 @@ def fvattn_attention_recall(importance, kv_idx, kv_cnt, recall, N: int, block: i
     return recall
 
 
+def fvattn_lvsa_lists(grid: Grid, window: int, period: int, step: int, kv_idx, kv_cnt, head_work,
+                      workspace, stream=None):
+    """LVSA window + rotating global-frame lists for every (b, h) of kv_cnt's [B,H,nb] shape."""
+    _need_cuda(kv_idx, kv_cnt, head_work, workspace)
+    B, H = kv_cnt.shape[:2]
+    _check(_lib.fvattn_lvsa_lists(B, H, ctypes.byref(grid), int(window), int(period), int(step),
+                                  _ptr(kv_idx), _ptr(kv_cnt), _ptr(head_work), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream)),
+           "fvattn_lvsa_lists")
+    return kv_idx, kv_cnt, head_work
+
+
+def fvattn_hilbert_table(grid_thw, block: int = 128, device="cuda", stream=None) -> torch.Tensor:
+    """Hilbert-curve order of grid (T, Hh, W): int32 [N] with table[pos] = raster index."""
+    T, Hh, W = grid_thw
+    g = Grid(T, Hh, W, 1, 1, 1, block, FVATTN_ORDER_TILES, None)
+    N = T * Hh * W
+    table = torch.empty(N, dtype=torch.int32, device=device)
+    ws = alloc_workspace(fvattn_workspace_bytes(FVATTN_OP_HILBERT, 1, 1, N, 64, block), device)
+    _check(_lib.fvattn_hilbert_table(ctypes.byref(g), _ptr(table), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)),
+           "fvattn_hilbert_table")
+    torch.cuda.current_stream(device).synchronize() if stream is None else stream.synchronize()
+    return table
+
+
 def fvattn_workspace_status(workspace, stream=None) -> int:
     """Synchronize the stream and return the status word the kernels recorded."""
     return int(_lib.fvattn_workspace_status(_ptr(workspace), _stream(stream)))
@@ -254,11 +297,16 @@ class FVAttnPath:
     ``__call__(q, k, v)`` takes [B,H,N,d] tensors in original token order and
     returns the attention output [B,H,N,d] in original order: route (which
     also permutes q and k), permute v, block-sparse attention, inverse permute.
-    ``dense=True`` runs the dense kernel instead of routing.
+    ``dense=True`` runs the dense kernel instead of routing. ``order="hilbert"``
+    orders blocks along the Hilbert curve (the table is built once here) instead
+    of 3-D tiles.
     """
 
-    def __init__(self, B, H, grid, tile, block, d, dtype, p, k_min, device="cuda"):
-        self.grid = Grid.make(grid, tile, block)
+    def __init__(self, B, H, grid, tile, block, d, dtype, p, k_min, device="cuda", order="tiles"):
+        if order not in ("tiles", "hilbert"):
+            raise ValueError(f"unknown block order {order!r}")
+        table = fvattn_hilbert_table(grid, block, device) if order == "hilbert" else None
+        self.grid = Grid.make(grid, tile, block, table=table)
         self.B, self.H, self.d = B, H, d
         self.N, self.nb = self.grid.N, self.grid.nb
         self.npad = self.nb * block

@@ -1,6 +1,7 @@
 // api.cu -- the extern "C" entry points of libfvattn.so (declared in
 // include/fvattn.h): host-side validation, workspace layout, TMA tensor maps
 // and kernel dispatch. No entry point allocates device memory.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cudaTypedefs.h>
@@ -32,6 +33,13 @@ cudaError_t launch_block_importance(const float* blse, const float* lse, const i
                                     int* status, cudaStream_t st);
 cudaError_t launch_attention_recall(const float* importance, const int* kv_idx, const int* kv_cnt,
                                     int BH, int nb, float* recall, int* status, cudaStream_t st);
+cudaError_t launch_lvsa_lists(const TileGeom& g, int N, int bs, int window, int per, int step,
+                              int BH, int* kv_idx, int* kv_cnt, unsigned long long* head_work,
+                              uint32_t* frames, cudaStream_t st);
+cudaError_t launch_hilbert_table(int T, int Hh, int W, int* table, unsigned long long* keys,
+                                 cudaStream_t st);
+int hilbert_bits(int extent);
+int next_pow2(int n);
 }  // namespace fvattn
 
 namespace {
@@ -41,6 +49,8 @@ using fvattn::kWsHeaderBytes;
 
 constexpr int kMaxBlocks = 4096;   // nb limit (route rows live in shared memory)
 constexpr int kMaxHeads = 4096;    // B*H limit (the work planner sorts heads in shared memory)
+constexpr int kMaxFrames = 1024;   // LVSA frame bitmasks hold 32 words
+constexpr size_t kLvsaBlockBytes = 128;   // one frame bitmask per block in the LVSA workspace
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 bool valid_dtype(fvattn_dtype dt) { return dt == FVATTN_BF16 || dt == FVATTN_FP32; }
@@ -132,13 +142,21 @@ bool make_row_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t bo
 fvattn_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA; }
 
 fvattn::TileGeom geom_of(const fvattn_grid* g) {
-  return fvattn::TileGeom{g->T, g->Hh, g->W, g->tt, g->th, g->tw};
+  return fvattn::TileGeom{g->T, g->Hh, g->W, g->tt, g->th, g->tw,
+                          g->order == FVATTN_ORDER_TABLE ? g->table : nullptr};
 }
 
 bool valid_grid(const fvattn_grid* g, int N) {
   if (!g) return false;
-  if (g->T < 1 || g->Hh < 1 || g->W < 1 || g->tt < 1 || g->th < 1 || g->tw < 1) return false;
+  if (g->T < 1 || g->Hh < 1 || g->W < 1) return false;
   if (!valid_block(g->block)) return false;
+  if (g->order == FVATTN_ORDER_TILES) {
+    if (g->tt < 1 || g->th < 1 || g->tw < 1) return false;
+  } else if (g->order == FVATTN_ORDER_TABLE) {
+    if (!g->table || !aligned(g->table, 4)) return false;
+  } else {
+    return false;
+  }
   const long long n = static_cast<long long>(g->T) * g->Hh * g->W;
   return n == N;
 }
@@ -222,6 +240,9 @@ size_t fvattn_workspace_bytes(fvattn_op op, int B, int H, int N, int d, int bloc
     case FVATTN_OP_SPARSE_FWD: return sparse_ws(B, H, N, block).total;
     case FVATTN_OP_DENSE_FWD: return kWsHeaderBytes;
     case FVATTN_OP_DIAG: return kWsHeaderBytes;
+    case FVATTN_OP_LVSA: return kWsHeaderBytes + align_up(num_blocks(N, block) * kLvsaBlockBytes, 256);
+    case FVATTN_OP_HILBERT:
+      return kWsHeaderBytes + align_up(static_cast<size_t>(fvattn::next_pow2(N)) * 8, 256);
   }
   return 0;
 }
@@ -333,6 +354,51 @@ fvattn_status fvattn_attention_recall(const float* importance, const int32_t* kv
   if (cudaMemsetAsync(workspace, 0, kWsHeaderBytes, st) != cudaSuccess) return FVATTN_ERR_CUDA;
   return from_cuda(fvattn::launch_attention_recall(importance, kv_idx, kv_cnt, B * H,
                                                    num_blocks(N, block), recall, &hdr->status, st));
+}
+
+fvattn_status fvattn_lvsa_lists(int B, int H, const fvattn_grid* grid, int window, int period,
+                                int step, int32_t* kv_idx, int32_t* kv_cnt, int64_t* head_work,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  if (!grid || !kv_idx || !kv_cnt || !head_work) return FVATTN_ERR_INVALID_ARG;
+  if (!aligned(kv_idx, 4) || !aligned(kv_cnt, 4) || !aligned(head_work, 8))
+    return FVATTN_ERR_INVALID_ARG;
+  const long long n = static_cast<long long>(grid->T) * grid->Hh * grid->W;
+  if (n < 1 || n > (1ll << 30)) return FVATTN_ERR_INVALID_ARG;
+  const int N = static_cast<int>(n);
+  if (!valid_grid(grid, N) || !valid_sizes(B, H, N, 64, grid->block)) return FVATTN_ERR_INVALID_ARG;
+  if (grid->T > kMaxFrames || window < 0 || period < 1) return FVATTN_ERR_INVALID_ARG;
+  const size_t need = fvattn_workspace_bytes(FVATTN_OP_LVSA, B, H, N, 64, grid->block);
+  const fvattn_status wst = check_ws(workspace, workspace_bytes, need);
+  if (wst != FVATTN_OK) return wst;
+  auto st = static_cast<cudaStream_t>(stream);
+  auto base = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(base, 0, kWsHeaderBytes, st) != cudaSuccess) return FVATTN_ERR_CUDA;
+  if (cudaMemsetAsync(head_work, 0, sizeof(int64_t) * B * H, st) != cudaSuccess)
+    return FVATTN_ERR_CUDA;
+  return from_cuda(fvattn::launch_lvsa_lists(
+      geom_of(grid), N, grid->block, window, period, step, B * H, kv_idx, kv_cnt,
+      reinterpret_cast<unsigned long long*>(head_work),
+      reinterpret_cast<uint32_t*>(base + kWsHeaderBytes), st));
+}
+
+fvattn_status fvattn_hilbert_table(const fvattn_grid* grid, int32_t* table, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  if (!grid || !table || !aligned(table, 4)) return FVATTN_ERR_INVALID_ARG;
+  if (grid->T < 1 || grid->Hh < 1 || grid->W < 1 || !valid_block(grid->block))
+    return FVATTN_ERR_INVALID_ARG;
+  const long long n = static_cast<long long>(grid->T) * grid->Hh * grid->W;
+  if (n > static_cast<long long>(kMaxBlocks) * grid->block) return FVATTN_ERR_INVALID_ARG;
+  const int N = static_cast<int>(n);
+  const int b = fvattn::hilbert_bits(std::max(grid->T, std::max(grid->Hh, grid->W)));
+  if (3 * b + fvattn::hilbert_bits(N) > 64) return FVATTN_ERR_UNSUPPORTED;
+  const size_t need = fvattn_workspace_bytes(FVATTN_OP_HILBERT, 1, 1, N, 64, grid->block);
+  const fvattn_status wst = check_ws(workspace, workspace_bytes, need);
+  if (wst != FVATTN_OK) return wst;
+  auto st = static_cast<cudaStream_t>(stream);
+  auto base = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(base, 0, kWsHeaderBytes, st) != cudaSuccess) return FVATTN_ERR_CUDA;
+  return from_cuda(fvattn::launch_hilbert_table(
+      grid->T, grid->Hh, grid->W, table, reinterpret_cast<unsigned long long*>(base + kWsHeaderBytes), st));
 }
 
 fvattn_status fvattn_workspace_status(const void* workspace, void* stream) {

@@ -31,6 +31,7 @@ __host__ __device__ __forceinline__ size_t align_up(size_t v, size_t a) {
 // tile has a closed form and so does the inverse map used here.
 struct TileGeom {
   int T, Hh, W, tt, th, tw;
+  const int* table;   // non-null: explicit order (table[pos] = raster index), e.g. Hilbert
 };
 
 // Original token index n = (t*Hh + y)*W + x of the token at permuted position pos.
@@ -53,6 +54,14 @@ __host__ __device__ __forceinline__ int tile_source_index(int pos, const TileGeo
   const int dy = rem / sx;
   const int dx = rem - dy * sx;
   return ((ti * g.tt + dt) * g.Hh + (yi * g.th + dy)) * g.W + (xi * g.tw + dx);
+}
+
+// Source row of permuted position pos (< N): the explicit table when there is
+// one, else the tile map. A table entry outside [0, N) gives -1 (row skipped).
+__device__ __forceinline__ int source_index(int pos, int N, const TileGeom& g) {
+  if (!g.table) return tile_source_index(pos, g);
+  const int s = __ldg(g.table + pos);
+  return (s >= 0 && s < N) ? s : -1;
 }
 
 __device__ __forceinline__ void record_status(int* status_word, int code) {

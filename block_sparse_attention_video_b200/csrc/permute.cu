@@ -1,4 +1,5 @@
-// permute.cu -- 3-D tile permutation of token rows [FVAttn §3.1] and the fused
+// permute.cu -- block-order permutation of token rows (3-D tiles, or an explicit
+// table such as the Hilbert order) [FVAttn §3.1] and the fused
 // gather + block-mean pooling pass of the routing front end [FVAttn §3.1:
 // block similarity from pooled Q/K].
 //
@@ -23,7 +24,7 @@ __global__ void __launch_bounds__(kCopyThreads)
   const int i = blockIdx.x - bh * nb;
   for (int r = threadIdx.x; r < bs; r += blockDim.x) {
     const int pos = i * bs + r;
-    src[r] = pos < N ? tile_source_index(pos, g) : -1;
+    src[r] = pos < N ? source_index(pos, N, g) : -1;
   }
   __syncthreads();
   const size_t orig_base = static_cast<size_t>(bh) * N;
@@ -98,7 +99,7 @@ __global__ void __launch_bounds__(kCopyThreads)
   const int i = blockIdx.x - bh * nb;
   for (int r = threadIdx.x; r < bs; r += blockDim.x) {
     const int pos = i * bs + r;
-    src[r] = pos < N ? tile_source_index(pos, g) : -1;
+    src[r] = pos < N ? source_index(pos, N, g) : -1;
   }
   __syncthreads();
   const size_t orig_base = static_cast<size_t>(bh) * N;

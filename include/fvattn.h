@@ -23,12 +23,15 @@
  * Diagnostic of mask quality, from statistics the attention kernels record:
  *   fvattn_block_importance  exact block importance   [GSRS §5.3, §A.2, §A.3]
  *   fvattn_attention_recall  attention recall of a mask            [GSRS §3.2]
+ * A second, static mask generator for the same attention kernel:
+ *   fvattn_lvsa_lists  local window + rotating global frames        [LVSA §3]
  *
  * Conventions (every entry point):
  *   - Tensors are dense, row-major, on the current CUDA device. A token row of
  *     d elements is contiguous. Shapes are given in the comments as [B,H,N,d].
  *   - N = T*Hh*W tokens in raster (t, y, x) order. nb = ceil(N/block) blocks;
- *     Npad = nb*block. "Permuted" tensors are [B,H,Npad,d] in tile order with
+ *     Npad = nb*block. "Permuted" tensors are [B,H,Npad,d] in the grid's block
+ *     order (3-D tiles, or an explicit table such as the Hilbert order) with
  *     the last Npad-N rows zero (written by fvattn_route / fvattn_permute).
  *   - The caller owns every buffer, including the workspace; the library never
  *     allocates or frees device memory and keeps no global state beyond a
@@ -75,18 +78,31 @@ typedef enum {
   FVATTN_FP32 = 1  /* SIMT path only (fp32 arithmetic throughout)           */
 } fvattn_dtype;
 
-/* Latent video grid and tiling [FVAttn §3.1, read as 3-D tiles]. */
+/* Block order of the token sequence [FVAttn §3.1; GSRS §A.6]. */
+typedef enum {
+  FVATTN_ORDER_TILES = 0, /* 3-D tiles (tt, th, tw), closed-form map          */
+  FVATTN_ORDER_TABLE = 1  /* explicit table, e.g. from fvattn_hilbert_table   */
+} fvattn_order;
+
+/* Latent video grid and block order. */
 typedef struct {
-  int T, Hh, W;   /* grid extents; N = T*Hh*W                               */
-  int tt, th, tw; /* tile extents (>= 1); edge tiles may be partial          */
-  int block;      /* tokens per block: 64 or 128                            */
+  int T, Hh, W;        /* grid extents; N = T*Hh*W                                  */
+  int tt, th, tw;      /* tile extents (>= 1; FVATTN_ORDER_TILES); edge tiles may be
+                          partial                                                   */
+  int block;           /* tokens per block: 64 or 128                               */
+  int order;           /* fvattn_order                                              */
+  const int32_t* table;/* FVATTN_ORDER_TABLE: device [N], table[pos] = raster index
+                          (t*Hh + y)*W + x of the token at permuted position pos; a
+                          permutation of [0, N) (entries outside it are skipped)    */
 } fvattn_grid;
 
 typedef enum {
   FVATTN_OP_ROUTE = 0,
   FVATTN_OP_SPARSE_FWD = 1,
   FVATTN_OP_DENSE_FWD = 2,
-  FVATTN_OP_DIAG = 3      /* fvattn_block_importance, fvattn_attention_recall */
+  FVATTN_OP_DIAG = 3,     /* fvattn_block_importance, fvattn_attention_recall */
+  FVATTN_OP_LVSA = 4,     /* fvattn_lvsa_lists */
+  FVATTN_OP_HILBERT = 5   /* fvattn_hilbert_table */
 } fvattn_op;
 
 /* Workspace bytes needed by `op` for these sizes (0 if the sizes are invalid).
@@ -94,13 +110,15 @@ typedef enum {
  * word, cleared at the start of every call that takes it. */
 FVATTN_API size_t fvattn_workspace_bytes(fvattn_op op, int B, int H, int N, int d, int block);
 
-/* 3-D tile permutation [FVAttn §3.1].
+/* Block-order permutation [FVAttn §3.1; GSRS §A.6].
  * inverse == 0: x [B,H,N,d] (original order) -> y [B,H,Npad,d] (tile order,
  *               pad rows zeroed).
  * inverse != 0: x [B,H,Npad,d] (tile order)  -> y [B,H,N,d] (original order,
  *               pad rows dropped).
- * Token at grid (t,y,x) moves to position pos(t,y,x): tiles in raster order
- * over the tile grid, raster order inside a tile. x and y must not overlap.
+ * FVATTN_ORDER_TILES: the token at grid (t,y,x) moves to position pos(t,y,x):
+ * tiles in raster order over the tile grid, raster order inside a tile.
+ * FVATTN_ORDER_TABLE: position pos holds the token grid->table[pos].
+ * x and y must not overlap.
  * d in {64, 128}; dtype BF16 or FP32. Bit-exact copy. */
 FVATTN_API fvattn_status fvattn_permute(const void* x, void* y, int B, int H, int N, int d,
                              fvattn_dtype dtype, const fvattn_grid* grid,
@@ -211,6 +229,41 @@ FVATTN_API fvattn_status fvattn_attention_recall(const float* importance, const 
                                                  const int32_t* kv_cnt, int B, int H, int N,
                                                  int block, float* recall, void* workspace,
                                                  size_t workspace_bytes, void* stream);
+
+/* Hilbert-curve token order of grid (T, Hh, W) [FVAttn §3.1; GSRS §A.6], for
+ * FVATTN_ORDER_TABLE grids. Tokens are ordered by their index on the 3-D
+ * Hilbert curve over (t, y, x) of the smallest cube of side 2^b holding the
+ * grid (b = bits of max(T, Hh, W)); the index is Skilling's ("Programming the
+ * Hilbert curve", 2004) with t as the first axis. table [N] int32 (device) gets
+ * table[pos] = raster index of the pos-th token along the curve. Built once per
+ * grid (one key pass, a bitonic sort of next_pow2(N) 64-bit keys, one gather).
+ * Uses only T, Hh, W and block of `grid`. Needs 3b + bits(N) <= 64
+ * (FVATTN_ERR_UNSUPPORTED otherwise). Workspace:
+ * fvattn_workspace_bytes(FVATTN_OP_HILBERT, 1, 1, N, 64, block). */
+FVATTN_API fvattn_status fvattn_hilbert_table(const fvattn_grid* grid, int32_t* table,
+                                              void* workspace, size_t workspace_bytes,
+                                              void* stream);
+
+/* KV block lists of the LVSA static pattern [LVSA §3], in the layout that
+ * fvattn_route produces and fvattn_sparse_fwd consumes.
+ * Frames: query frame t attends A(t) = G ∪ W(t) with
+ *   G    = { g in [0,T) : g = step (mod period) }  (equidistant global frames,
+ *          rotated by the denoising step);
+ *   W(t) = [t-window, t+window] clipped to [0,T), then expanded until
+ *          |A(t)| = |G| + min(2*window+1, T-|G|) for every t: each pass adds the
+ *          current deficit, ceil(deficit/2) frames after t and the rest before
+ *          t, a clipped side handing its share to the other side.
+ * Blocks: blocks of the tile-ordered sequence of `grid` (as fvattn_permute);
+ * key block j is listed for query block i when a valid token of i lies in a
+ * frame tq and a valid token of j in a frame of A(tq).
+ * Outputs, the same for every (b,h): kv_idx [B,H,nb,nb] (ascending at entries
+ * [0,cnt)), kv_cnt [B,H,nb], head_work [B,H] = sum_i cnt.
+ * T <= 1024, window >= 0, period >= 1, any step. Workspace:
+ * fvattn_workspace_bytes(FVATTN_OP_LVSA, B, H, N, d, block) for any valid d. */
+FVATTN_API fvattn_status fvattn_lvsa_lists(int B, int H, const fvattn_grid* grid, int window,
+                                           int period, int step, int32_t* kv_idx, int32_t* kv_cnt,
+                                           int64_t* head_work, void* workspace,
+                                           size_t workspace_bytes, void* stream);
 
 /* Synchronizes `stream` and returns the status word that the kernels of the
  * last call using `workspace` recorded (FVATTN_OK if none). */

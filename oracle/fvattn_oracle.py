@@ -152,17 +152,19 @@ def head_work(cnt: np.ndarray) -> np.ndarray:
     return np.asarray(cnt, dtype=np.int64).sum(axis=-1)
 
 
-def route(q, k, grid, bs: int, p: float, k_min: int, scale: float | None = None):
+def route(q, k, grid, bs: int, p: float, k_min: int, scale: float | None = None, perm=None):
     """Routing front end for q, k ``[B, H, N, d]`` in original token order.
 
-    Steps: tile permutation, block-mean pooling of Q and K, block scores, and
+    Steps: tile permutation (or the explicit token order ``perm``, e.g. the
+    Hilbert order, when given), block-mean pooling of Q and K, block scores, and
     per-row Top-p with the Top-k floor. Returns a dict with ``perm``,
     ``qbar``, ``kbar``, ``scores`` (fp64 [B,H,nb,nb]), ``order`` (int64
     [B,H,nb,nb]), ``cnt`` (int64 [B,H,nb]) and ``head_work`` (int64 [B,H]).
     Heads are processed one at a time to bound memory.
     """
     T, Hh, W, tt, th, tw = grid
-    perm = tile_order(T, Hh, W, tt, th, tw)
+    if perm is None:
+        perm = tile_order(T, Hh, W, tt, th, tw)
     B, H, N, d = q.shape
     if N != len(perm):
         raise ValueError("N must equal T*Hh*W")

@@ -177,3 +177,69 @@ def test_attention_recall_rejects(kw, status):
 def test_diag_workspace_is_the_status_word():
     assert F.fvattn_workspace_bytes(F.FVATTN_OP_DIAG, 1, 2, 256, 64, 64) == 256
     assert F.fvattn_workspace_bytes(F.FVATTN_OP_DIAG, 1, 2, 256, 32, 64) == 0
+
+
+def _lvsa(grid=None, B=1, H=2, window=1, period=3, step=0, idx=FAKE, cnt=FAKE, hw=FAKE, ws=FAKE,
+          ws_bytes=1 << 20):
+    g = grid if grid is not None else _grid()
+    return F._lib.fvattn_lvsa_lists(B, H, ctypes.byref(g), window, period, step, idx, cnt, hw, ws,
+                                    ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw, status", [
+    (dict(idx=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(hw=FAKE + 4), F.FVATTN_ERR_INVALID_ARG),        # head_work must be 8-byte aligned
+    (dict(window=-1), F.FVATTN_ERR_INVALID_ARG),
+    (dict(period=0), F.FVATTN_ERR_INVALID_ARG),
+    (dict(B=0), F.FVATTN_ERR_INVALID_ARG),
+    (dict(grid=_grid(T=1100, Hh=1, W=1, th=1, tw=1)), F.FVATTN_ERR_INVALID_ARG),   # more than 1024 frames
+    (dict(grid=_grid(block=32)), F.FVATTN_ERR_INVALID_ARG),
+    (dict(ws=None), F.FVATTN_ERR_WORKSPACE),
+    (dict(ws_bytes=256), F.FVATTN_ERR_WORKSPACE),
+])
+def test_lvsa_rejects(kw, status):
+    assert _lvsa(**kw) == status
+
+
+def test_lvsa_workspace_holds_one_frame_mask_per_block():
+    nb = 4
+    assert F.fvattn_workspace_bytes(F.FVATTN_OP_LVSA, 1, 2, 256, 64, 64) == 256 + 512
+    assert F.fvattn_workspace_bytes(F.FVATTN_OP_LVSA, 1, 2, 256 * 64, 128, 64) == 256 + 256 * 128
+    assert nb * 128 == 512
+
+
+def test_grid_order_is_validated():
+    g = _grid()
+    g.order = F.FVATTN_ORDER_TABLE                      # a table order without a table
+    assert F._lib.fvattn_permute(FAKE, FAKE * 4, 1, 2, 256, 64, F.FVATTN_FP32, ctypes.byref(g), 0,
+                                 None) == F.FVATTN_ERR_INVALID_ARG
+    g.table = FAKE + 2                                  # misaligned table
+    assert F._lib.fvattn_permute(FAKE, FAKE * 4, 1, 2, 256, 64, F.FVATTN_FP32, ctypes.byref(g), 0,
+                                 None) == F.FVATTN_ERR_INVALID_ARG
+    g.order = 7                                         # unknown order
+    assert F._lib.fvattn_permute(FAKE, FAKE * 4, 1, 2, 256, 64, F.FVATTN_FP32, ctypes.byref(g), 0,
+                                 None) == F.FVATTN_ERR_INVALID_ARG
+    assert ctypes.sizeof(F.Grid) == 40
+
+
+def _hilbert(grid=None, table=FAKE, ws=FAKE, ws_bytes=1 << 30):
+    g = grid if grid is not None else _grid()
+    return F._lib.fvattn_hilbert_table(ctypes.byref(g), table, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw, status", [
+    (dict(table=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(table=FAKE + 2), F.FVATTN_ERR_INVALID_ARG),
+    (dict(grid=_grid(T=0)), F.FVATTN_ERR_INVALID_ARG),
+    (dict(grid=_grid(block=96)), F.FVATTN_ERR_INVALID_ARG),
+    (dict(grid=_grid(T=4097, Hh=1, W=128)), F.FVATTN_ERR_INVALID_ARG),          # more than 4096 blocks
+    (dict(grid=_grid(T=1, Hh=1, W=1 << 19, block=128)), F.FVATTN_ERR_UNSUPPORTED),  # 3*19 + 19 key bits
+    (dict(ws=None), F.FVATTN_ERR_WORKSPACE),
+    (dict(ws_bytes=1024), F.FVATTN_ERR_WORKSPACE),
+])
+def test_hilbert_table_rejects(kw, status):
+    assert _hilbert(**kw) == status
+
+
+def test_hilbert_workspace_holds_the_padded_keys():
+    assert F.fvattn_workspace_bytes(F.FVATTN_OP_HILBERT, 1, 1, 75600, 64, 128) == 256 + (1 << 17) * 8
