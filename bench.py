@@ -47,8 +47,7 @@ METRIC = "sparse attn ms/call & effective TFLOP/s (Wan-14B 720p shape) vs own de
 # the kernel source they were taken on. They are reported only while the source
 # is unchanged; after any change the traffic is unknown and reported as null.
 ATTN_TRAFFIC = {
-    "wan14b-720p": {"bytes": 2.54e9 + 764.24e6, "src": "d8063faaf0ab5a25"},
-    "wan14b-480p": {"bytes": 1.023992e9 + 321.768704e6, "src": "d8063faaf0ab5a25"},
+    "wan14b-720p": {"bytes": 2.53e9 + 763.56e6, "src": "bdaacdca49693a3a"},
 }
 ATTN_SRC = os.path.join(ROOT, "block_sparse_attention_video_b200", "csrc", "attn_sm100.cu")
 
@@ -415,36 +414,34 @@ def run_fvattn(args):
         diag = run_diag(F, w, path, stream, args.warmup,
                         lvsa_lists=(lvsa.pop("_lists") if lvsa is not None else None))
 
-    # ---- e2e through the public API with pinned host buffers
+    # ---- e2e through the public API with pinned host buffers: every step uploads its
+    # q, k, v and downloads its output; HostPipeline overlaps the copies of
+    # neighbouring steps with the kernels of the current one.
     e2e = None
     if not args.no_e2e:
         hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
         hout = torch.empty(path.out.shape, dtype=path.out.dtype).pin_memory()
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-
-        def e2e_step():
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            out = path(dq, dk, dv)
-            hout.copy_(out, non_blocking=True)
-
-        for _ in range(max(1, args.warmup)):
-            e2e_step()
+        pipe = F.HostPipeline(path)
+        pipe.run([(hq, hk, hv)] * max(1, args.warmup), [hout] * max(1, args.warmup))
         torch.cuda.synchronize()
-        e_steps = max(2, args.steps // 2)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e_steps = max(2, args.steps)
+        a = torch.cuda.Event(enable_timing=True)
         _barrier(dist)
         a.record(stream)
-        for _ in range(e_steps):
-            e2e_step()
+        end_ev = pipe.run([(hq, hk, hv)] * e_steps, [hout] * e_steps, start_event=a)
+        b = torch.cuda.Event(enable_timing=True)
         b.record(stream)
         torch.cuda.synchronize()
         _barrier(dist)
         ms_e2e = _max_over_ranks(dist, a.elapsed_time(b) / e_steps)
+        if F.fvattn_workspace_status(path.ws_attn) != F.FVATTN_OK:
+            raise RuntimeError("kernel status word set in the e2e run")
         in_bytes = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
         e2e = {"value": world * eff / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms_e2e,
-               "h2d_bytes_per_step": int(in_bytes), "d2h_bytes_per_step": int(hout.numel() * hout.element_size())}
+               "h2d_bytes_per_step": int(in_bytes), "d2h_bytes_per_step": int(hout.numel() * hout.element_size()),
+               "steps": e_steps, "overlap": "copies of neighbouring steps overlap the current step's kernels"}
+        del pipe
+        torch.cuda.empty_cache()
 
     if rank != 0:
         if dist is not None:

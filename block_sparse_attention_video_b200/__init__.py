@@ -12,7 +12,9 @@ Entry points carry the C names: ``fvattn_permute``, ``fvattn_route``,
 ``fvattn_hilbert_table``,
 ``fvattn_workspace_bytes``, ``fvattn_workspace_status``. ``FVAttnPath`` strings them into the full per-call
 path (route -> permute V -> block-sparse attention -> inverse permute) over
-buffers it allocates once with torch.
+buffers it allocates once with torch; ``HostPipeline`` runs it over a sequence
+of calls with pinned host inputs and outputs, overlapping the copies of
+neighbouring calls with the kernels of the current one.
 """
 
 from __future__ import annotations
@@ -339,7 +341,9 @@ class FVAttnPath:
             fvattn_sparse_fwd(self.qp, self.kp, self.vp, self.op, self.kv_idx, self.kv_cnt,
                               self.N, self.block, self.ws_attn)
 
-    def __call__(self, q, k, v, dense=False):
+    def __call__(self, q, k, v, dense=False, out=None):
+        """q, k, v [B,H,N,d] (original order) -> attention output [B,H,N,d] in ``out``
+        (default: a buffer owned by the path, overwritten by the next call)."""
         if dense:
             fvattn_permute(q, self.qp, self.grid)
             fvattn_permute(k, self.kp, self.grid)
@@ -347,5 +351,73 @@ class FVAttnPath:
             self.route(q, k)
         fvattn_permute(v, self.vp, self.grid)
         self.attend(dense=dense)
-        fvattn_permute(self.op, self.out, self.grid, inverse=True)
-        return self.out
+        dst = self.out if out is None else out
+        fvattn_permute(self.op, dst, self.grid, inverse=True)
+        return dst
+
+
+class HostPipeline:
+    """Runs an FVAttnPath over a sequence of calls whose q, k, v live in pinned host
+    memory and whose outputs go back to pinned host memory, with the copies of
+    neighbouring calls overlapping the kernels of the current one.
+
+    Two device input sets and two output buffers alternate. Uploads run on one
+    copy stream, downloads on another, and the kernels on the current stream.
+    Events order them: call i's kernels wait for its upload; its download waits
+    for its kernels; the upload of call i+2 waits until call i's kernels have
+    read the shared input set; call i+2's kernels wait until call i's download
+    has read the shared output buffer.
+    """
+
+    def __init__(self, path: FVAttnPath, dense=False):
+        self.path = path
+        self.dense = dense
+        dev = path.qp.device
+        shp = (path.B, path.H, path.N, path.d)
+        self.inp = [tuple(torch.empty(shp, dtype=path.dtype, device=dev) for _ in range(3)) for _ in range(2)]
+        self.outp = [torch.empty(shp, dtype=path.dtype, device=dev) for _ in range(2)]
+        self.up = torch.cuda.Stream(device=dev)
+        self.down = torch.cuda.Stream(device=dev)
+        self._ev = lambda: torch.cuda.Event()
+        self.done_read = [None, None]     # kernels of the last call on slot s have read its inputs
+        self.done_down = [None, None]     # download of the last call on slot s has read its output
+
+    def run(self, host_qkv, host_out, start_event=None):
+        """host_qkv: sequence of (q, k, v) pinned CPU tensors; host_out: sequence of
+        pinned CPU tensors (may repeat). Enqueues every call; returns the event
+        recorded on the current stream after the last download."""
+        comp = torch.cuda.current_stream(self.path.qp.device)
+        if start_event is not None:
+            self.up.wait_event(start_event)
+            self.down.wait_event(start_event)
+        last = None
+        for i, ((hq, hk, hv), ho) in enumerate(zip(host_qkv, host_out)):
+            s = i & 1
+            dq, dk, dv = self.inp[s]
+            with torch.cuda.stream(self.up):
+                if self.done_read[s] is not None:
+                    self.up.wait_event(self.done_read[s])
+                dq.copy_(hq, non_blocking=True)
+                dk.copy_(hk, non_blocking=True)
+                dv.copy_(hv, non_blocking=True)
+                ev_in = self._ev()
+                ev_in.record(self.up)
+            comp.wait_event(ev_in)
+            if self.done_down[s] is not None:
+                comp.wait_event(self.done_down[s])
+            self.path(dq, dk, dv, dense=self.dense, out=self.outp[s])
+            ev_k = self._ev()
+            ev_k.record(comp)
+            self.done_read[s] = ev_k
+            with torch.cuda.stream(self.down):
+                self.down.wait_event(ev_k)
+                ho.copy_(self.outp[s], non_blocking=True)
+                ev_d = self._ev()
+                ev_d.record(self.down)
+            self.done_down[s] = ev_d
+            last = ev_d
+        if last is not None:
+            comp.wait_event(last)
+        end = self._ev()
+        end.record(comp)
+        return end

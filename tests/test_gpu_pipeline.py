@@ -1,0 +1,36 @@
+"""GPU: HostPipeline (pinned host inputs and outputs, copies of neighbouring calls
+overlapping the current call's kernels) gives, call by call, exactly the output of
+FVAttnPath on device inputs (the kernels are deterministic per work unit)."""
+
+import pytest
+import torch
+
+import synthetic as S
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import block_sparse_attention_video_b200 as F
+
+
+@pytest.mark.parametrize("dense", [False, True])
+def test_host_pipeline_matches_per_call_results(dense):
+    w = S.WORKLOADS["wan1.3b-480p"]
+    calls = [S.make_qkv(w.replace(seed=w.seed + 100 * i), device="cuda") for i in range(3)]
+    path = F.FVAttnPath(w.B, w.H, w.grid, w.tile, w.block, w.d, torch.bfloat16, w.p, w.k_min)
+    want = [path(q, k, v, dense=dense).clone() for (q, k, v) in calls]
+    host_in = [tuple(x.cpu().pin_memory() for x in qkv) for qkv in calls]
+    host_out = [torch.empty(want[0].shape, dtype=want[0].dtype).pin_memory() for _ in calls]
+    pipe = F.HostPipeline(path, dense=dense)
+    pipe.run(host_in, host_out)
+    torch.cuda.synchronize()
+    assert F.fvattn_workspace_status(path.ws_attn) == F.FVATTN_OK
+    for i in range(len(calls)):
+        assert torch.equal(host_out[i], want[i].cpu()), i
+    # a second run reuses the same slots
+    host_out2 = [torch.zeros_like(h) for h in host_out]
+    host_out2 = [h.pin_memory() for h in host_out2]
+    pipe.run(host_in[::-1], host_out2)
+    torch.cuda.synchronize()
+    for i in range(len(calls)):
+        assert torch.equal(host_out2[i], want[::-1][i].cpu()), i
