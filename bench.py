@@ -148,17 +148,25 @@ class ClockSampler:
                 "power_w_max": max(r[3] for r in rows)}
 
 
-def _dist_setup(n_gpus):
+def _dist_setup(n_gpus, backend="nccl"):
+    """One process per GPU (torchrun env). The data path has no collective: the
+    group only carries the barriers and the max over ranks of the timings.
+    backend "gloo" (CPU tests) leaves the CUDA device alone."""
+    import datetime
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    timeout = datetime.timedelta(seconds=120)
     if world > 1:
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
-                                timeout=__import__("datetime").timedelta(seconds=120))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", device_id=torch.device("cuda", local), timeout=timeout)
+        else:
+            dist.init_process_group(backend, timeout=timeout)
         return dist, rank, world, local
-    torch.cuda.set_device(local)
+    if backend == "nccl":
+        torch.cuda.set_device(local)
     return None, 0, 1, local
 
 
@@ -167,10 +175,10 @@ def _barrier(dist):
         dist.barrier()
 
 
-def _max_over_ranks(dist, v: float) -> float:
+def _max_over_ranks(dist, v: float, device="cuda") -> float:
     if dist is None:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -335,12 +343,17 @@ def run_diag(F, w, path, stream, warmup, lvsa_lists=None):
     return out
 
 
+def replica_workload(w, rank: int):
+    """Each rank runs an independent call of the same shape on its own inputs."""
+    return w.replace(seed=w.seed + 1000 * rank)
+
+
 def run_fvattn(args):
     import block_sparse_attention_video_b200 as F
     dist, rank, world, local = _dist_setup(args.gpus)
     w = S.WORKLOADS[args.workload]
     dev = torch.device("cuda", local)
-    q, k, v = S.make_qkv(w.replace(seed=w.seed + 1000 * rank), device=dev)
+    q, k, v = S.make_qkv(replica_workload(w, rank), device=dev)
     path = F.FVAttnPath(w.B, w.H, w.grid, w.tile, w.block, w.d, torch.bfloat16, w.p, w.k_min, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -540,7 +553,8 @@ def run_reference(args):
         flops += one_step((args.warmup + s_) % w.H)
     dt = time.perf_counter() - t0
     tf = flops / dt / 1e12
-    line = {"metric": METRIC, "value": tf, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+    line = {"metric": METRIC, "value": tf, "unit": "TFLOP/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+            "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",

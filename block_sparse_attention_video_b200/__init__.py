@@ -355,6 +355,27 @@ class FVAttnPath:
         fvattn_permute(self.op, dst, self.grid, inverse=True)
         return dst
 
+    def capture_graph(self, q, k, v, dense=False, out=None):
+        """Captures one whole call on the given tensors into a CUDA graph (the
+        library allocates nothing and never synchronizes the host inside a call,
+        so every step is capturable). ``graph.replay()`` re-runs it on whatever q,
+        k, v hold at that time. Returns (graph, output tensor)."""
+        dst = self.out if out is None else out
+        return _capture(self, q, k, v, dense, dst), dst
+
+
+def _capture(path, q, k, v, dense, out):
+    dev = path.qp.device
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):          # first launches (kernel attributes) outside the capture
+        path(q, k, v, dense=dense, out=out)
+    torch.cuda.current_stream(dev).wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        path(q, k, v, dense=dense, out=out)
+    return graph
+
 
 class HostPipeline:
     """Runs an FVAttnPath over a sequence of calls whose q, k, v live in pinned host

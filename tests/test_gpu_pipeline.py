@@ -34,3 +34,23 @@ def test_host_pipeline_matches_per_call_results(dense):
     torch.cuda.synchronize()
     for i in range(len(calls)):
         assert torch.equal(host_out2[i], want[::-1][i].cpu()), i
+
+
+@pytest.mark.parametrize("dense", [False, True])
+def test_cuda_graph_replay_matches_eager(dense):
+    w = S.WORKLOADS["wan1.3b-480p"]
+    q, k, v = S.make_qkv(w, device="cuda")
+    path = F.FVAttnPath(w.B, w.H, w.grid, w.tile, w.block, w.d, torch.bfloat16, w.p, w.k_min)
+    out = torch.empty_like(q)
+    graph, res = path.capture_graph(q, k, v, dense=dense, out=out)
+    for shift in (7, 19):
+        q2, k2, v2 = S.make_qkv(w.replace(seed=w.seed + shift), device="cuda")
+        want = path(q2, k2, v2, dense=dense).clone()
+        q.copy_(q2)
+        k.copy_(k2)
+        v.copy_(v2)
+        res.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert F.fvattn_workspace_status(path.ws_attn) == F.FVATTN_OK
+        assert torch.equal(res, want), shift
