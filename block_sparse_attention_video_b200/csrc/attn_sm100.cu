@@ -31,12 +31,15 @@
 // S1(k), and finally PV0(last) PV1(last): the exponentials of one slot overlap
 // the other slot's MMAs.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512).
-// P (bf16, two per 32-bit column) overwrites the first BN/2 columns of S and is
+// P (bf16, two per 32-bit column) overwrites the first 64 columns of S and is
 // the A operand of the P.V MMA straight from TMEM.
-// Shared memory: Q0, Q1 (32 KB each) and a 128 KB K/V ring (4 x 32 KB stages for
-// BN = 128, 8 x 16 KB for BN = 64), tiles stored as two 128-byte-swizzled halves
-// of 64 columns, as TMA writes them. K-major descriptors for Q and K, MN-major
-// for V.
+// Shared memory: Q0, Q1 (32 KB each) and a 128 KB K/V ring of 4 x 32 KB stages
+// of 128 key rows, stored as two 128-byte-swizzled halves of 64 columns, as TMA
+// writes them. A step is 128 keys: one 128-token block, or (BN = 64) two
+// consecutive union entries whose 64-row tiles fill the two row halves of the
+// stage, so every S MMA is N = 128 and every P.V is K = 128 whatever BN is; the
+// softmax masks, sums and records each 64-key half of such a step by its own
+// entry. K-major descriptors for Q and K, MN-major for V.
 //
 // Scheduling [FVAttn §2.2, §3.2: per-head work differs widely across heads]:
 // units are claimed in an order prepared on the device (heads by descending
@@ -71,13 +74,19 @@ constexpr float kLn2 = 0.6931471805599453f;
 #endif
 constexpr int kPolyEvery = FVATTN_POLY_EVERY;
 
+// A step covers 128 keys: one 128-token block, or two consecutive union entries
+// of 64-token blocks whose K (V) tiles are loaded into the two 64-row halves of
+// one 128-row stage. Every step is then an N = 128 S MMA and a K = 128 P.V.
 template <int BN>
 struct Tile {
-  static constexpr int kKVBytes = BN * HD * 2;
-  static constexpr int kKVHalf = BN * 128;
+  static constexpr int kStepKeys = 128;
+  static constexpr int kBPS = kStepKeys / BN;              // union entries per step
+  static constexpr int kKVBytes = kStepKeys * HD * 2;      // 32 KB stage
+  static constexpr int kKVHalf = kStepKeys * 128;          // one 64-column half of a stage
+  static constexpr int kSubBytes = BN * 128;               // one entry's rows within a half
   static constexpr int kStages = kRingBytes / kKVBytes;
-  static constexpr int kGroup = kUnitRows / BN;   // query blocks per unit
-  static constexpr uint32_t kIdescQK = umma_idesc_bf16(128, BN, false);
+  static constexpr int kGroup = kUnitRows / BN;            // query blocks per unit
+  static constexpr uint32_t kIdescQK = umma_idesc_bf16(128, kStepKeys, false);
   static constexpr uint32_t kIdescPV = umma_idesc_bf16(128, HD, true);
 };
 
@@ -250,8 +259,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(sm.q[X] + kQHalfBytes, &tm_q, &sm.q_full[X], 64, row0 + X * 128);
           ++qn[X];
         }
-        for (int k = 0; ok && k < x.cnt; ++k) {
-          const int kvrow = x.bh * P.npad + static_cast<int>(entry_at<BN>(x, k, P) & 0xFFFFu) * BN;
+        const int ns = (x.cnt + T::kBPS - 1) / T::kBPS;
+        for (int k = 0; ok && k < ns; ++k) {
+          int kvrow[T::kBPS];
+#pragma unroll
+          for (int h = 0; h < T::kBPS; ++h) {
+            // past the list's end (odd count): repeat the step's first block; its
+            // half of the S tile is masked by the softmax warps
+            const int idx = T::kBPS * k + h < x.cnt ? T::kBPS * k + h : T::kBPS * k;
+            kvrow[h] = x.bh * P.npad + static_cast<int>(entry_at<BN>(x, idx, P) & 0xFFFFu) * BN;
+          }
 #pragma unroll
           for (int t = 0; t < 2; ++t) {     // K(k) then V(k)
             const int s = it % kStages;
@@ -259,8 +276,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(&sm.kv_full[s], T::kKVBytes);
             uint8_t* dst = sm.kv + s * T::kKVBytes;
             const CUtensorMap* tm = t == 0 ? &tm_k : &tm_v;
-            tma_load_2d(dst, tm, &sm.kv_full[s], 0, kvrow);
-            tma_load_2d(dst + T::kKVHalf, tm, &sm.kv_full[s], 64, kvrow);
+#pragma unroll
+            for (int h = 0; h < T::kBPS; ++h) {
+              tma_load_2d(dst + h * T::kSubBytes, tm, &sm.kv_full[s], 0, kvrow[h]);
+              tma_load_2d(dst + T::kKVHalf + h * T::kSubBytes, tm, &sm.kv_full[s], 64, kvrow[h]);
+            }
             ++it;
           }
         }
@@ -286,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++un;
         const Unit x = decode_unit<BN>(u, P);
         if (x.cnt == 0) break;
-        const int cnt = x.cnt;
+        const int cnt = (x.cnt + T::kBPS - 1) / T::kBPS;   // steps of 128 keys
         auto kv_ready = [&](int o) -> bool {
           return mbar_wait(&sm.kv_full[o % kStages], (o / kStages) & 1, abort_flag, P.status);
         };
@@ -309,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         };
         auto pv_op = [&](int X, int k) -> bool {  // O_X += P_X V(k), V(k) already waited on
-          // P arrives in two halves (key columns [0, BN/2) and [BN/2, BN)); the
+          // P arrives in two halves (key columns [0, 64) and [64, 128)); the
           // first half's MMAs run while the softmax warps finish the second.
           const uint32_t va = kv_addr + ((base + 2 * k + 1) % kStages) * T::kKVBytes;
 #pragma unroll
@@ -317,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(&sm.p_full[X][h], pn[X] & 1, abort_flag, P.status)) return false;
             tc_fence_after();
 #pragma unroll
-            for (int kk = h * (BN / 32); kk < (h + 1) * (BN / 32); ++kk) {
+            for (int kk = h * (T::kStepKeys / 32); kk < (h + 1) * (T::kStepKeys / 32); ++kk) {
               umma_ts(tmem + 256 + X * 128, tmem + X * 128 + kk * 8,
                       umma_desc_sw128(va + kk * 2048, T::kKVHalf, 1024), T::kIdescPV,
                       (k > 0 || kk > 0) ? 1u : 0u);
@@ -354,7 +374,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   regs_inc<kRegsSoftmax>();
   {
     // ------------------------------------------------------------ softmax / epilogue
-    constexpr int NC = BN / 32;          // 32-column chunks of S
+    constexpr int NC = T::kStepKeys / 32;   // 32-column chunks of S
+    constexpr int BPS = T::kBPS;            // union entries per step
+    constexpr int CPE = NC / BPS;           // chunks per entry
     const int X = warp >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
@@ -376,29 +398,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit x = decode_unit<BN>(u, P);
       if (x.cnt == 0) break;
       if (!(X == 0 ? x.slot[0] : x.slot[1])) continue;
+      const int ns = (x.cnt + BPS - 1) / BPS;
+      const int qrow = x.grp * kUnitRows + X * 128 + row;   // row within the head
       float m_run = -FLT_MAX;
       float l_run = 0.f;
       bool have = false;
       bool ok = true;
-      uint32_t e_next = entry_at<BN>(x, 0, P);
+      // Entries of the next step, read ahead; past the list's end, 0 (no member).
+      uint32_t e_next[BPS];
+#pragma unroll
+      for (int h = 0; h < BPS; ++h) e_next[h] = h < x.cnt ? entry_at<BN>(x, h, P) : 0u;
 #pragma unroll 1
-      for (int k = 0; k < x.cnt; ++k) {
+      for (int k = 0; k < ns; ++k) {
         if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[X], sn & 1, abort_flag, P.status))) { ok = false; break; }
         ++sn;
         tc_fence_after();
-        const uint32_t e = e_next;
-        if (k + 1 < x.cnt) e_next = entry_at<BN>(x, k + 1, P);   // hide the list read behind this block
-        if ((e >> (16 + qb)) & 1u) {
+        uint32_t e[BPS];
+        bool mem[BPS];
+        bool any_mem = false;
+#pragma unroll
+        for (int h = 0; h < BPS; ++h) {
+          e[h] = e_next[h];
+          const int idx = BPS * (k + 1) + h;
+          if (k + 1 < ns) e_next[h] = idx < x.cnt ? entry_at<BN>(x, idx, P) : 0u;
+          mem[h] = (e[h] >> (16 + qb)) & 1u;     // warp-uniform: a warp's rows share qb
+          any_mem |= mem[h];
+        }
+        if (any_mem) {
           uint32_t s[NC][32];
 #pragma unroll
           for (int c = 0; c < NC; ++c) tmem_ld32(tS + c * 32, s[c]);
           tmem_wait_ld();
-          if (static_cast<int>(e & 0xFFFFu) == P.nb - 1 && tail < BN) {
+          // Keys this row does not attend: the other half's block when the row's
+          // query block did not select it (or the pad half of an odd step), and
+          // the keys past N of the last block.
 #pragma unroll
-            for (int c = 0; c < NC; ++c)
+          for (int c = 0; c < NC; ++c) {
+            const int h = c / CPE;
+            const int kbase = (c % CPE) * 32;     // first key of the chunk within its block
+            if (!mem[h]) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) s[c][i] = __float_as_uint(-INFINITY);
+            } else if (static_cast<int>(e[h] & 0xFFFFu) == P.nb - 1 && tail < kbase + 32) {
 #pragma unroll
               for (int i = 0; i < 32; ++i)
-                if (c * 32 + i >= tail) s[c][i] = __float_as_uint(-INFINITY);
+                if (kbase + i >= tail) s[c][i] = __float_as_uint(-INFINITY);
+            }
           }
           // Row max: 8 independent chains of 3-input max (exact in any order).
           float mx8[8];
@@ -436,14 +481,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (need) m_run = m_new;
             }
           }
-          // x = s * scale*log2(e) - m and the row sum in packed fp32x2 arithmetic.
+          // x = s * scale*log2(e) - m and the row sums in packed fp32x2 arithmetic.
           // Each half of P is published as soon as it is in TMEM.
           const float2 sl2x2 = make_float2(sl2, sl2);
           const float2 negm = make_float2(-m_run, -m_run);
-          float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          float2 lc[NC];
 #pragma unroll
           for (int c = 0; c < NC; ++c) {
             uint32_t pk[16];
+            float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float2 xv = __ffma2_rn(
@@ -460,6 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               ls[i & 1] = __fadd2_rn(ls[i & 1], make_float2(p0, p1));
               pk[i] = pack_bf16x2(p0, p1);
             }
+            lc[c] = __fadd2_rn(ls[0], ls[1]);
             tmem_st16(tS + c * 16, pk);
             if (c == NC / 2 - 1 || c == NC - 1) {
               tmem_wait_st();
@@ -468,15 +515,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (lane == 0) mbar_arrive(&sm.p_full[X][c == NC - 1 ? 1 : 0]);
             }
           }
-          const float l_blk = (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
-          l_run += l_blk;
-          // Block log-sum-exp of this row over this key block [GSRS §5.3]: the
-          // exponentials above are relative to m_run, so it is m_run + log2 of
-          // their sum, converted to the natural base.
-          if (P.blse) {
-            const int qrow = x.grp * kUnitRows + X * 128 + row;
-            if (qrow < P.npad)
-              P.blse[(static_cast<size_t>(x.bh) * P.nb + (e & 0xFFFFu)) * P.npad + qrow] =
+#pragma unroll
+          for (int h = 0; h < BPS; ++h) {
+            float l_blk = 0.f;
+#pragma unroll
+            for (int c = h * CPE; c < (h + 1) * CPE; ++c) l_blk += lc[c].x + lc[c].y;
+            l_run += l_blk;
+            // Block log-sum-exp of this row over this key block [GSRS §5.3]: the
+            // exponentials are relative to m_run, so it is m_run + log2 of their
+            // sum, converted to the natural base.
+            if (P.blse && mem[h] && qrow < P.npad)
+              P.blse[(static_cast<size_t>(x.bh) * P.nb + (e[h] & 0xFFFFu)) * P.npad + qrow] =
                   (m_run + __log2f(l_blk)) * kLn2;
           }
         } else {
@@ -501,7 +550,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Rows past the head's last block (the second half of a 64-token-block
       // tile at the end of a head) are not stored; the TMEM loads stay
       // warp-collective.
-      const int qrow = x.grp * kUnitRows + X * 128 + row;   // row within the head
       const bool store = qrow < P.npad;
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
       const size_t grow = static_cast<size_t>(x.bh) * P.npad + qrow;
