@@ -243,3 +243,17 @@ def test_hilbert_table_rejects(kw, status):
 
 def test_hilbert_workspace_holds_the_padded_keys():
     assert F.fvattn_workspace_bytes(F.FVATTN_OP_HILBERT, 1, 1, 75600, 64, 128) == 256 + (1 << 17) * 8
+
+
+def test_empty_inputs_are_rejected_before_any_launch():
+    # N = 0 tokens (an empty grid) at every entry point that takes N
+    g0 = _grid(T=0)
+    assert F._lib.fvattn_permute(FAKE, FAKE * 4, 1, 2, 0, 64, F.FVATTN_FP32, ctypes.byref(g0), 0,
+                                 None) == F.FVATTN_ERR_INVALID_ARG
+    assert _route(grid=g0, N=0) == F.FVATTN_ERR_INVALID_ARG
+    assert _sparse(N=0) == F.FVATTN_ERR_INVALID_ARG
+    assert F._lib.fvattn_dense_fwd(FAKE, FAKE, FAKE, FAKE, None, None, 1, 2, 0, 64, F.FVATTN_FP32, 64,
+                                   0.125, FAKE, 1 << 20, None) == F.FVATTN_ERR_INVALID_ARG
+    assert _lvsa(grid=g0) == F.FVATTN_ERR_INVALID_ARG
+    assert _hilbert(grid=g0) == F.FVATTN_ERR_INVALID_ARG
+    assert F.fvattn_workspace_bytes(F.FVATTN_OP_SPARSE_FWD, 1, 2, 0, 64, 64) == 0
