@@ -191,7 +191,7 @@ def fvattn_route(q, k, grid: Grid, p: float, k_min: int, kv_idx, kv_cnt, head_wo
 def fvattn_route_noalloc(q, k, grid: Grid, p: float, k_min: int, kv_idx, kv_cnt, head_work,
                          qp_out=None, kp_out=None, stream=None):
     """fvattn_route without a workspace, for callers that cannot allocate device
-    memory where they route; the library's static 32 MiB device scratch is used
+    memory where they route; the library's static 96 MiB device scratch is used
     instead (calls that overlap on the GPU race on it)."""
     _need_cuda(q, k, kv_idx, kv_cnt, head_work, qp_out, kp_out)
     B, H, N, d = q.shape

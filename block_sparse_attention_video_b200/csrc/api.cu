@@ -14,8 +14,8 @@ cudaError_t launch_permute(const void* x, void* y, int BH, int N, int d, int esi
 cudaError_t launch_gather_pool(const void* q, const void* k, void* qp, void* kp, float* qbar,
                                float* kbar, int BH, int N, int d, bool bf16, int bs,
                                const TileGeom& g, cudaStream_t st);
-int route_select_rows_per_warp(int nb, int d);
-cudaError_t launch_route_select(const float* qbar, const float* kbar, int BH, int nb, int d,
+size_t route_scores_bytes(int BH, int nb);
+cudaError_t launch_route_select(const float* qbar, const float* kbar, float* S, int BH, int nb, int d,
                                 float scale, float p, int k_min, int* kv_idx, int* kv_cnt,
                                 unsigned long long* head_work, int* status, cudaStream_t st);
 cudaError_t launch_attn_simt(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -70,15 +70,19 @@ bool valid_sizes(int B, int H, int N, int d, int block) {
 int num_blocks(int N, int block) { return (N + block - 1) / block; }
 
 // ------------------------------------------------------------- workspace layout
+// Route workspace: status header, the pooled q and k means, and the block score
+// matrix [B*H, nb, nb] fp32 that the selection kernel reads back.
 struct RouteWs {
-  size_t qbar, kbar, total;
+  size_t qbar, kbar, scores, total;
 };
 RouteWs route_ws(int B, int H, int N, int d, int block) {
-  const size_t bars = static_cast<size_t>(B) * H * num_blocks(N, block) * d * sizeof(float);
+  const int nb = num_blocks(N, block);
+  const size_t bars = static_cast<size_t>(B) * H * nb * d * sizeof(float);
   RouteWs w;
   w.qbar = kWsHeaderBytes;
   w.kbar = w.qbar + align_up(bars, 256);
-  w.total = w.kbar + align_up(bars, 256);
+  w.scores = w.kbar + align_up(bars, 256);
+  w.total = w.scores + align_up(fvattn::route_scores_bytes(B * H, nb), 256);
   return w;
 }
 
@@ -279,7 +283,6 @@ fvattn_status fvattn_route(const void* q, const void* k, int B, int H, int N, in
   if (!(p > 0.f && p <= 1.f) || k_min < 1) return FVATTN_ERR_INVALID_ARG;
   const int block = grid->block;
   const int nb = num_blocks(N, block);
-  if (fvattn::route_select_rows_per_warp(nb, d) == 0) return FVATTN_ERR_UNSUPPORTED;
   const RouteWs w = route_ws(B, H, N, d, block);
   const fvattn_status wst = check_ws(workspace, workspace_bytes, w.total);
   if (wst != FVATTN_OK) return wst;
@@ -297,7 +300,8 @@ fvattn_status fvattn_route(const void* q, const void* k, int B, int H, int N, in
                                              dtype == FVATTN_BF16, block, geom_of(grid), st);
   if (e != cudaSuccess) return FVATTN_ERR_CUDA;
   const float scale = 1.0f / std::sqrt(static_cast<float>(d));
-  e = fvattn::launch_route_select(qbar, kbar, BH, nb, d, scale, p, k_min, kv_idx, kv_cnt,
+  float* scores = reinterpret_cast<float*>(base + w.scores);
+  e = fvattn::launch_route_select(qbar, kbar, scores, BH, nb, d, scale, p, k_min, kv_idx, kv_cnt,
                                   reinterpret_cast<unsigned long long*>(head_work), &hdr->status,
                                   st);
   return from_cuda(e);

@@ -5,18 +5,19 @@
 // plugin inside an inference engine that owns all device memory and offers no
 // scratch buffer, or a latency-critical loop where cudaMalloc would synchronize
 // the device and stall it. This entry point takes no workspace. Its scratch
-// (the status word and the pooled q/k block means that fvattn_route keeps in
-// its workspace) lives in the file-scope device array below, which every GPU
+// (the status word, the pooled q/k block means and the block score matrix that
+// fvattn_route keeps in its workspace) lives in the file-scope device array below, which every GPU
 // that loads the library holds until the process exits.
 //
 // Limits and sharing:
-//   - At most kScratchBytes (32 MiB) of scratch: sizes whose route workspace
+//   - At most kScratchBytes (96 MiB) of scratch: sizes whose route workspace
 //     (fvattn_workspace_bytes(FVATTN_OP_ROUTE, ...)) is larger are rejected with
 //     FVATTN_ERR_WORKSPACE before anything is launched. The Wan-14B 720p shape
-//     (40 heads, 591 blocks, d = 128) needs 24.2 MB and fits.
+//     (40 heads, 591 blocks, d = 128) needs 80.1 MB (block means 24.2 MB, block
+//     scores 55.9 MB) and fits.
 //   - Every call on a device uses the same array and leaves its contents for
 //     the next call. The router clears the status word at the start of each
-//     call and overwrites the block means completely, so no stale value is
+//     call and overwrites the block means and scores completely, so no stale value is
 //     read. Calls whose kernels overlap on the GPU (concurrent streams, or
 //     several host threads) race on the array: keep them ordered.
 //   - The array's device address is looked up with cudaGetSymbolAddress on the
@@ -30,7 +31,7 @@
 
 namespace {
 
-constexpr size_t kScratchBytes = static_cast<size_t>(32) << 20;
+constexpr size_t kScratchBytes = static_cast<size_t>(96) << 20;
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char fvattn_route_scratch[kScratchBytes];

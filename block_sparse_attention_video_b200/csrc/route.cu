@@ -1,19 +1,24 @@
 // route.cu -- block scores, softmax and Top-p / Top-k-floor selection
 // [FVAttn §2.1, §2.2 Eq. (1), §3.1; GSRS §5.2, §5.3, §A.4].
 //
-// One CTA owns ROWS = 8*RP query blocks of one (b, h):
-//   1. scores S[r][j] = scale * qbar_r . kbar_j for every key block j, fp32, by
-//      a register-tiled SIMT product (kbar streamed through shared memory in
-//      chunks of 128 key blocks); the score rows stay in shared memory;
-//   2. one warp per row: max-subtracted softmax (expf, fixed-order warp sums),
+// Two kernels, each at high occupancy:
+//   1. block_scores_kernel: S[b,h,i,j] = scale * qbar_i . kbar_j for every pair
+//      of blocks, fp32, as a 64 x 64 tiled SIMT product (4 x 4 outputs per
+//      thread, both tiles staged k-major in shared memory); S goes to the route
+//      workspace.
+//   2. select_rows_kernel: one warp per (b, h, query block) row, the row staged
+//      in shared memory: max-subtracted softmax (expf, fixed-order warp sums),
 //      then the Top-p cut found without sorting: the largest value v* with
 //      F(v*) = sum_{s_j >= v*} s_j >= p, located by bisection on the bit
 //      pattern of non-negative floats (the computed F is monotone in v because
 //      fp32 sums of non-negative terms are monotone in each term); ties at v*
-//      are taken in block-index order until the sum reaches p. If the Top-k
-//      floor is larger, the k_min-th largest value is found the same way on
-//      counts. The selected blocks are compacted in ascending index order with
-//      warp ballots, the count is stored and added to the per-head work.
+//      are taken in block-index order until the sum reaches p. F only changes at
+//      the row's values, so v* is one of them: the bisection also counts the
+//      values at or above each bound and stops as soon as one distinct value is
+//      left between them, which is then v*. If the Top-k floor is larger, the
+//      k_min-th largest value is found the same way on counts. The selected
+//      blocks are compacted in ascending index order with warp ballots, the
+//      count is stored and added to the per-head work.
 // Deterministic: every sum has a fixed order.
 #include <cfloat>
 
@@ -22,7 +27,6 @@
 namespace fvattn {
 
 constexpr int kRouteThreads = 256;
-constexpr int kKeyChunk = 128;
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -51,9 +55,19 @@ __device__ __forceinline__ float mass_at_least(const float* s, int nb, float thr
 }
 
 __device__ __forceinline__ int count_at_least(const float* s, int nb, float thr, int lane) {
-  int c = 0;
-  for (int j = lane; j < nb; j += 32) c += s[j] >= thr ? 1 : 0;
-  return warp_sum_int(c);
+  unsigned c = 0u;
+  for (int j = lane; j < nb; j += 32) c += s[j] >= thr ? 1u : 0u;
+  return static_cast<int>(__reduce_add_sync(0xffffffffu, c));
+}
+
+// The only value of the row in [lo, hi) (the caller knows there is exactly one).
+__device__ __forceinline__ uint32_t only_value_below(const float* s, int nb, uint32_t hi, int lane) {
+  unsigned m = 0u;
+  for (int j = lane; j < nb; j += 32) {
+    const unsigned b = __float_as_uint(s[j]);
+    if (b < hi) m = max(m, b);
+  }
+  return __reduce_max_sync(0xffffffffu, m);
 }
 
 // One importance row (already scaled logits in s[0..nb)), one warp.
@@ -90,10 +104,16 @@ __device__ void select_row(float* s, int nb, float p, int k_min, int* __restrict
       n_p = nb;
     } else {
       uint32_t lo = 0u, hi = 0x3F800001u;          // F(lo) >= p > F(hi)
-      while (hi - lo > 1u) {
+      int c_lo = nb, c_hi = 0;                     // values at or above lo, hi
+      while (hi - lo > 1u && c_lo - c_hi > 1) {
         const uint32_t mid = lo + ((hi - lo) >> 1);
-        if (mass_at_least(s, nb, __uint_as_float(mid), lane) >= p) lo = mid; else hi = mid;
+        const float fm = mass_at_least(s, nb, __uint_as_float(mid), lane);
+        const int cm = count_at_least(s, nb, __uint_as_float(mid), lane);
+        if (fm >= p) { lo = mid; c_lo = cm; } else { hi = mid; c_hi = cm; }
       }
+      // One value left in [lo, hi): it is v*. (Otherwise lo and hi are adjacent
+      // floats and v* = lo.)
+      if (c_lo - c_hi == 1) lo = only_value_below(s, nb, hi, lane);
       vstar = __uint_as_float(lo);
       float sgt = 0.f;
       int ceq = 0;
@@ -119,10 +139,13 @@ __device__ void select_row(float* s, int nb, float p, int k_min, int* __restrict
       take_eq = cnt - cgt;
     } else {
       uint32_t lo = 0u, hi = 0x3F800001u;          // count(lo) >= cnt > count(hi)
-      while (hi - lo > 1u) {
+      int c_lo = nb, c_hi = 0;
+      while (hi - lo > 1u && c_lo - c_hi > 1) {
         const uint32_t mid = lo + ((hi - lo) >> 1);
-        if (count_at_least(s, nb, __uint_as_float(mid), lane) >= cnt) lo = mid; else hi = mid;
+        const int cm = count_at_least(s, nb, __uint_as_float(mid), lane);
+        if (cm >= cnt) { lo = mid; c_lo = cm; } else { hi = mid; c_hi = cm; }
       }
+      if (c_lo - c_hi == 1) lo = only_value_below(s, nb, hi, lane);
       thr = __uint_as_float(lo);
       int gt = 0;
       for (int j = lane; j < nb; j += 32) gt += s[j] > thr ? 1 : 0;
@@ -152,122 +175,108 @@ __device__ void select_row(float* s, int nb, float p, int k_min, int* __restrict
   }
 }
 
-template <int RP>
-__global__ void __launch_bounds__(kRouteThreads)
-    route_select_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar, int nb,
-                        int d, float scale, float p, int k_min, int* __restrict__ kv_idx,
-                        int* __restrict__ kv_cnt, unsigned long long* __restrict__ head_work,
-                        int* status) {
-  constexpr int ROWS = 8 * RP;
-  extern __shared__ float4 smem_f4[];
-  float* sm = reinterpret_cast<float*>(smem_f4);
-  const int ds = d + 4;
-  float* qs = sm;                      // ROWS x ds
-  float* ks = qs + ROWS * ds;          // kKeyChunk x ds
-  float* S = ks + kKeyChunk * ds;      // ROWS x nb
+constexpr int kTile = 64;        // score tile: 64 query blocks x 64 key blocks
+constexpr int kTilePad = kTile + 4;
 
-  const int bh = blockIdx.y;
-  const int i0 = blockIdx.x * ROWS;
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
+// S tile = scale * Qtile . Ktile^T over d; 16 x 16 threads, 4 x 4 outputs each.
+__global__ void __launch_bounds__(kRouteThreads)
+    block_scores_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar, int nb, int d,
+                        float scale, float* __restrict__ S) {
+  extern __shared__ float4 smem_f4[];
+  float* qs = reinterpret_cast<float*>(smem_f4);   // [d][kTilePad], k-major
+  float* ks = qs + d * kTilePad;                   // [d][kTilePad]
+  const int bh = blockIdx.z;
+  const int i0 = blockIdx.y * kTile, j0 = blockIdx.x * kTile;
   const float* qb = qbar + static_cast<size_t>(bh) * nb * d;
   const float* kb = kbar + static_cast<size_t>(bh) * nb * d;
   const int d4 = d >> 2;
-
-  for (int e = tid; e < ROWS * d4; e += kRouteThreads) {
-    const int r = e / d4, c = (e - r * d4) * 4;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i0 + r < nb) v = *reinterpret_cast<const float4*>(qb + static_cast<size_t>(i0 + r) * d + c);
-    *reinterpret_cast<float4*>(qs + r * ds + c) = v;
-  }
-  for (int j0 = 0; j0 < nb; j0 += kKeyChunk) {
-    __syncthreads();
-    for (int e = tid; e < kKeyChunk * d4; e += kRouteThreads) {
-      const int r = e / d4, c = (e - r * d4) * 4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j0 + r < nb) v = *reinterpret_cast<const float4*>(kb + static_cast<size_t>(j0 + r) * d + c);
-      *reinterpret_cast<float4*>(ks + r * ds + c) = v;
-    }
-    __syncthreads();
-    float acc[RP][4];
-#pragma unroll
-    for (int a = 0; a < RP; ++a)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
-    for (int kk = 0; kk < d; kk += 4) {
-      float4 kv[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) kv[c] = *reinterpret_cast<const float4*>(ks + (lane + 32 * c) * ds + kk);
-#pragma unroll
-      for (int a = 0; a < RP; ++a) {
-        const float4 qv = *reinterpret_cast<const float4*>(qs + (warp * RP + a) * ds + kk);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float t = acc[a][c];
-          t = fmaf(qv.x, kv[c].x, t);
-          t = fmaf(qv.y, kv[c].y, t);
-          t = fmaf(qv.z, kv[c].z, t);
-          t = fmaf(qv.w, kv[c].w, t);
-          acc[a][c] = t;
-        }
-      }
-    }
-#pragma unroll
-    for (int a = 0; a < RP; ++a)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int j = j0 + lane + 32 * c;
-        if (j < nb) S[(warp * RP + a) * nb + j] = acc[a][c] * scale;
-      }
+  // rows of the tile are the fastest index so that the transposing stores hit distinct banks
+  for (int e = threadIdx.x; e < kTile * d4; e += kRouteThreads) {
+    const int r = e % kTile, c = (e / kTile) * 4;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (i0 + r < nb) a = *reinterpret_cast<const float4*>(qb + static_cast<size_t>(i0 + r) * d + c);
+    if (j0 + r < nb) b = *reinterpret_cast<const float4*>(kb + static_cast<size_t>(j0 + r) * d + c);
+    qs[(c + 0) * kTilePad + r] = a.x;
+    qs[(c + 1) * kTilePad + r] = a.y;
+    qs[(c + 2) * kTilePad + r] = a.z;
+    qs[(c + 3) * kTilePad + r] = a.w;
+    ks[(c + 0) * kTilePad + r] = b.x;
+    ks[(c + 1) * kTilePad + r] = b.y;
+    ks[(c + 2) * kTilePad + r] = b.z;
+    ks[(c + 3) * kTilePad + r] = b.w;
   }
   __syncthreads();
-  for (int a = 0; a < RP; ++a) {
-    const int r = warp * RP + a;
-    const int i = i0 + r;
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  float acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
+#pragma unroll 4
+  for (int kk = 0; kk < d; ++kk) {
+    const float4 qa = *reinterpret_cast<const float4*>(qs + kk * kTilePad + ty * 4);
+    const float4 kv = *reinterpret_cast<const float4*>(ks + kk * kTilePad + tx * 4);
+    const float qv[4] = {qa.x, qa.y, qa.z, qa.w};
+    const float kf[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(qv[a], kf[c], acc[a][c]);
+  }
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int i = i0 + ty * 4 + a;
     if (i >= nb) break;
-    const size_t row = static_cast<size_t>(bh) * nb + i;
-    select_row(S + r * nb, nb, p, k_min, kv_idx + row * nb, kv_cnt + row, head_work + bh,
-               status, lane);
+    float* row = S + (static_cast<size_t>(bh) * nb + i) * nb;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int j = j0 + tx * 4 + c;
+      if (j < nb) row[j] = acc[a][c] * scale;
+    }
   }
 }
 
-size_t route_select_smem_bytes(int rp, int nb, int d) {
-  return (static_cast<size_t>(8 * rp) * (d + 4) + static_cast<size_t>(kKeyChunk) * (d + 4) +
-          static_cast<size_t>(8 * rp) * nb) * sizeof(float);
+// One warp per row of S: stage the row in shared memory, then select.
+__global__ void __launch_bounds__(kRouteThreads)
+    select_rows_kernel(const float* __restrict__ S, int rows, int nb, float p, int k_min,
+                       int* __restrict__ kv_idx, int* __restrict__ kv_cnt,
+                       unsigned long long* __restrict__ head_work, int* status) {
+  extern __shared__ float4 smem_f4[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* srow = reinterpret_cast<float*>(smem_f4) + static_cast<size_t>(warp) * nb;
+  const int r = blockIdx.x * (kRouteThreads / 32) + warp;
+  if (r >= rows) return;
+  const float* src = S + static_cast<size_t>(r) * nb;
+  for (int j = lane; j < nb; j += 32) srow[j] = src[j];
+  __syncwarp();
+  const int bh = r / nb;
+  select_row(srow, nb, p, k_min, kv_idx + static_cast<size_t>(r) * nb, kv_cnt + r, head_work + bh,
+             status, lane);
 }
 
-int route_select_rows_per_warp(int nb, int d) {
-  constexpr size_t kBudget = 200 * 1024;
-  for (int rp : {4, 2, 1})
-    if (route_select_smem_bytes(rp, nb, d) <= kBudget) return rp;
-  return 0;
+size_t route_scores_bytes(int BH, int nb) {
+  return static_cast<size_t>(BH) * nb * nb * sizeof(float);
 }
 
-cudaError_t launch_route_select(const float* qbar, const float* kbar, int BH, int nb, int d,
+cudaError_t launch_route_select(const float* qbar, const float* kbar, float* S, int BH, int nb, int d,
                                 float scale, float p, int k_min, int* kv_idx, int* kv_cnt,
                                 unsigned long long* head_work, int* status, cudaStream_t st) {
-  const int rp = route_select_rows_per_warp(nb, d);
-  if (rp == 0) return cudaErrorInvalidValue;
-  const size_t smem = route_select_smem_bytes(rp, nb, d);
-  const dim3 grid((nb + 8 * rp - 1) / (8 * rp), BH);
-  cudaError_t e;
-  switch (rp) {
-    case 4:
-      e = cudaFuncSetAttribute(route_select_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      route_select_kernel<4><<<grid, kRouteThreads, smem, st>>>(qbar, kbar, nb, d, scale, p, k_min, kv_idx, kv_cnt, head_work, status);
-      break;
-    case 2:
-      e = cudaFuncSetAttribute(route_select_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      route_select_kernel<2><<<grid, kRouteThreads, smem, st>>>(qbar, kbar, nb, d, scale, p, k_min, kv_idx, kv_cnt, head_work, status);
-      break;
-    default:
-      e = cudaFuncSetAttribute(route_select_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      route_select_kernel<1><<<grid, kRouteThreads, smem, st>>>(qbar, kbar, nb, d, scale, p, k_min, kv_idx, kv_cnt, head_work, status);
-      break;
-  }
+  const size_t smem1 = static_cast<size_t>(2) * d * kTilePad * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(block_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem1));
+  if (e != cudaSuccess) return e;
+  const dim3 g1((nb + kTile - 1) / kTile, (nb + kTile - 1) / kTile, BH);
+  block_scores_kernel<<<g1, kRouteThreads, smem1, st>>>(qbar, kbar, nb, d, scale, S);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem2 = static_cast<size_t>(kRouteThreads / 32) * nb * sizeof(float);
+  e = cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem2));
+  if (e != cudaSuccess) return e;
+  const int rows = BH * nb;
+  const int warps = kRouteThreads / 32;
+  select_rows_kernel<<<(rows + warps - 1) / warps, kRouteThreads, smem2, st>>>(
+      S, rows, nb, p, k_min, kv_idx, kv_cnt, head_work, status);
   return cudaGetLastError();
 }
 

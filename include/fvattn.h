@@ -142,7 +142,9 @@ FVATTN_API fvattn_status fvattn_permute(const void* x, void* y, int B, int H, in
  *   kv_cnt    [B,H,nb] int32: cnt per query block.
  *   head_work [B,H] int64: sum_i cnt = nb * L_h of Eq. (1).
  * 0 < p <= 1, k_min >= 1, d in {64,128}, block in {64,128}, N = T*Hh*W,
- * nb <= 4096. Workspace: fvattn_workspace_bytes(FVATTN_OP_ROUTE, ...). */
+ * nb <= 4096. Workspace: fvattn_workspace_bytes(FVATTN_OP_ROUTE, ...): the
+ * status word, the pooled means (2 x B*H*nb*d fp32) and the block score matrix
+ * (B*H*nb*nb fp32). */
 FVATTN_API fvattn_status fvattn_route(const void* q, const void* k, int B, int H, int N, int d,
                            fvattn_dtype dtype, const fvattn_grid* grid, float p,
                            int k_min, void* qp_out, void* kp_out, int32_t* kv_idx,
@@ -154,8 +156,8 @@ FVATTN_API fvattn_status fvattn_route(const void* q, const void* k, int B, int H
  * cudaMalloc would synchronize the device). The pages have no counterpart to
  * this call; it exists only for how the library is embedded.
  * Same arguments and results as fvattn_route, minus the workspace: the scratch
- * is a library-owned static device array of 32 MiB that every GPU loading the
- * library keeps until exit. Sizes whose route workspace exceeds 32 MiB return
+ * is a library-owned static device array of 96 MiB that every GPU loading the
+ * library keeps until exit. Sizes whose route workspace exceeds 96 MiB return
  * FVATTN_ERR_WORKSPACE and launch nothing. All calls on a device share the
  * array, so calls that overlap on the GPU race; the first call on each device
  * looks up the array's address (do it before any stream capture). Nothing is
