@@ -398,7 +398,7 @@ def run_fvattn(args):
     attn_ms = [a.elapsed_time(b) for a, b in ev]
     ms_attn = sum(attn_ms) / len(attn_ms)
     ms_step_max = _max_over_ranks(dist, ms_step)
-    launches_per_step = 8   # gather_pool, route_select, permute V, plan x3, attention, inverse permute
+    launches_per_step = 9   # gather_pool, block scores, select rows, permute V, plan x3, attention, inverse
 
     # ---- the build's own dense kernel at the same shape
     dense_ms = []
