@@ -47,7 +47,7 @@ METRIC = "sparse attn ms/call & effective TFLOP/s (Wan-14B 720p shape) vs own de
 # the kernel source they were taken on. They are reported only while the source
 # is unchanged; after any change the traffic is unknown and reported as null.
 ATTN_TRAFFIC = {
-    "wan14b-720p": {"bytes": 2.53e9 + 763.56e6, "src": "bdaacdca49693a3a"},
+    "wan14b-720p": {"bytes": 2.54e9 + 763.87e6, "src": "619c7d8a8f916bed"},
 }
 ATTN_SRC = os.path.join(ROOT, "block_sparse_attention_video_b200", "csrc", "attn_sm100.cu")
 
@@ -568,6 +568,38 @@ def run_reference(args):
     return 0
 
 
+def run_sweep(args):
+    """The 720p sweep (p x k_min x block size): one JSON line per config with its
+    density, route and attention times and effective TFLOP/s (not the headline line)."""
+    import block_sparse_attention_video_b200 as F
+    _dist_setup(1)
+    base = S.WORKLOADS["wan14b-720p"]
+    q, k, v = S.make_qkv(base, device="cuda")
+    stream = torch.cuda.current_stream()
+    paths = {}
+    for w in S.sweep_workloads():
+        key = (w.block, w.tile)
+        if key not in paths:
+            paths.clear()
+            torch.cuda.empty_cache()
+            paths[key] = F.FVAttnPath(w.B, w.H, w.grid, w.tile, w.block, w.d, torch.bfloat16, w.p, w.k_min)
+        path = paths[key]
+        path.p, path.k_min = float(w.p), int(w.k_min)
+        route_ms = _median_ms(lambda: path.route(q, k), stream, args.warmup, 3)
+        F.fvattn_permute(v, path.vp, path.grid)
+        attn_ms = _median_ms(lambda: path.attend(), stream, args.warmup, 3)
+        if F.fvattn_workspace_status(path.ws_attn) != F.FVATTN_OK:
+            raise RuntimeError("kernel status word set in the sweep")
+        idx, cnt = path.kv_idx.cpu().numpy(), path.kv_cnt.cpu().numpy()
+        eff = effective_flops(idx, cnt, w.N, w.block, w.d)
+        hw = path.head_work.cpu().numpy().astype(np.float64)
+        print(json.dumps({"sweep": w.name, "block": w.block, "p": w.p, "k_min": w.k_min,
+                          "density": float(cnt.mean() / path.nb), "route_ms": route_ms, "attention_ms": attn_ms,
+                          "effective_tflops": eff / (attn_ms * 1e-3) / 1e12,
+                          "head_work_max_over_mean": float(hw.max() / hw.mean())}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -580,10 +612,14 @@ def main(argv=None):
     ap.add_argument("--no-diag", action="store_true", help="skip the GSRS block-importance diagnostic")
     ap.add_argument("--no-lvsa", action="store_true", help="skip the LVSA static-mask measurement")
     ap.add_argument("--no-hilbert", action="store_true", help="skip the Hilbert-order measurement")
+    ap.add_argument("--sweep", action="store_true",
+                    help="print the 720p p x k_min x block-size sweep (one JSON line per config) instead")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "fvattn":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.sweep:
+        return run_sweep(args)
     return run_reference(args) if args.impl == "reference" else run_fvattn(args)
 
 
