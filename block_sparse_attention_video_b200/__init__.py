@@ -8,7 +8,7 @@ fallback: importing it fails loudly if the library has not been built
 
 Entry points carry the C names: ``fvattn_permute``, ``fvattn_route``,
 ``fvattn_route_noalloc``, ``fvattn_sparse_fwd``, ``fvattn_dense_fwd``,
-``fvattn_block_importance``, ``fvattn_attention_recall``, ``fvattn_lvsa_lists``,
+``fvattn_block_importance``, ``fvattn_attention_recall``, ``fvattn_select_topp``, ``fvattn_lvsa_lists``,
 ``fvattn_hilbert_table``,
 ``fvattn_workspace_bytes``, ``fvattn_workspace_status``. ``FVAttnPath`` strings them into the full per-call
 path (route -> permute V -> block-sparse attention -> inverse permute) over
@@ -57,7 +57,7 @@ FVATTN_ORDER_TABLE = 1
 
 EXPORTED = ("fvattn_workspace_bytes", "fvattn_permute", "fvattn_route", "fvattn_route_noalloc",
             "fvattn_sparse_fwd", "fvattn_dense_fwd", "fvattn_block_importance", "fvattn_attention_recall",
-            "fvattn_lvsa_lists", "fvattn_hilbert_table",
+            "fvattn_select_topp", "fvattn_lvsa_lists", "fvattn_hilbert_table",
             "fvattn_workspace_status", "fvattn_status_string")
 
 
@@ -113,6 +113,9 @@ _lib.fvattn_block_importance.restype = _c_int
 _lib.fvattn_attention_recall.argtypes = [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int,
                                          _c_int, _c_void_p, _c_void_p, _c_size_t, _c_void_p]
 _lib.fvattn_attention_recall.restype = _c_int
+_lib.fvattn_select_topp.argtypes = [_c_void_p, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_void_p,
+                                    _c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_void_p]
+_lib.fvattn_select_topp.restype = _c_int
 _lib.fvattn_lvsa_lists.argtypes = [_c_int, _c_int, ctypes.POINTER(Grid), _c_int, _c_int, _c_int, _c_void_p,
                                    _c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_void_p]
 _lib.fvattn_lvsa_lists.restype = _c_int
@@ -253,6 +256,18 @@ def fvattn_attention_recall(importance, kv_idx, kv_cnt, recall, N: int, block: i
                                         workspace.numel() * workspace.element_size(), _stream(stream)),
            "fvattn_attention_recall")
     return recall
+
+
+def fvattn_select_topp(importance, N: int, block: int, p: float, k_min: int, kv_idx, kv_cnt, head_work,
+                       workspace, stream=None):
+    """Top-p + Top-k floor on importance rows [B,H,nb,nb] (the GSRS search over a candidate set)."""
+    _need_cuda(importance, kv_idx, kv_cnt, head_work, workspace)
+    B, H = kv_cnt.shape[:2]
+    _check(_lib.fvattn_select_topp(_ptr(importance), B, H, N, block, float(p), int(k_min), _ptr(kv_idx),
+                                   _ptr(kv_cnt), _ptr(head_work), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+           "fvattn_select_topp")
+    return kv_idx, kv_cnt, head_work
 
 
 def fvattn_lvsa_lists(grid: Grid, window: int, period: int, step: int, kv_idx, kv_cnt, head_work,

@@ -15,6 +15,9 @@ cudaError_t launch_gather_pool(const void* q, const void* k, void* qp, void* kp,
                                float* kbar, int BH, int N, int d, bool bf16, int bs,
                                const TileGeom& g, cudaStream_t st);
 size_t route_scores_bytes(int BH, int nb);
+cudaError_t launch_select_topp(const float* rows_in, int BH, int nb, float p, int k_min, int* kv_idx,
+                               int* kv_cnt, unsigned long long* head_work, int* status,
+                               cudaStream_t st);
 cudaError_t launch_route_select(const float* qbar, const float* kbar, float* S, int BH, int nb, int d,
                                 float scale, float p, int k_min, int* kv_idx, int* kv_cnt,
                                 unsigned long long* head_work, int* status, cudaStream_t st);
@@ -358,6 +361,26 @@ fvattn_status fvattn_attention_recall(const float* importance, const int32_t* kv
   if (cudaMemsetAsync(workspace, 0, kWsHeaderBytes, st) != cudaSuccess) return FVATTN_ERR_CUDA;
   return from_cuda(fvattn::launch_attention_recall(importance, kv_idx, kv_cnt, B * H,
                                                    num_blocks(N, block), recall, &hdr->status, st));
+}
+
+fvattn_status fvattn_select_topp(const float* importance, int B, int H, int N, int block, float p,
+                                int k_min, int32_t* kv_idx, int32_t* kv_cnt, int64_t* head_work,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  if (!importance || !kv_idx || !kv_cnt || !head_work) return FVATTN_ERR_INVALID_ARG;
+  if (!aligned(importance, 4) || !aligned(kv_idx, 4) || !aligned(kv_cnt, 4) || !aligned(head_work, 8))
+    return FVATTN_ERR_INVALID_ARG;
+  if (!valid_sizes(B, H, N, 64, block)) return FVATTN_ERR_INVALID_ARG;
+  if (!(p > 0.f && p <= 1.f) || k_min < 1) return FVATTN_ERR_INVALID_ARG;
+  const fvattn_status wst = check_ws(workspace, workspace_bytes, kWsHeaderBytes);
+  if (wst != FVATTN_OK) return wst;
+  auto st = static_cast<cudaStream_t>(stream);
+  auto hdr = static_cast<fvattn::WsHeader*>(workspace);
+  if (cudaMemsetAsync(workspace, 0, kWsHeaderBytes, st) != cudaSuccess) return FVATTN_ERR_CUDA;
+  if (cudaMemsetAsync(head_work, 0, sizeof(int64_t) * B * H, st) != cudaSuccess)
+    return FVATTN_ERR_CUDA;
+  return from_cuda(fvattn::launch_select_topp(importance, B * H, num_blocks(N, block), p, k_min, kv_idx,
+                                              kv_cnt, reinterpret_cast<unsigned long long*>(head_work),
+                                              &hdr->status, st));
 }
 
 fvattn_status fvattn_lvsa_lists(int B, int H, const fvattn_grid* grid, int window, int period,

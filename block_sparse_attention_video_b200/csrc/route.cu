@@ -71,21 +71,36 @@ __device__ __forceinline__ uint32_t only_value_below(const float* s, int nb, uin
 }
 
 // One importance row (already scaled logits in s[0..nb)), one warp.
+// With softmax == false the row already holds importances (non-negative,
+// summing to one over the evaluated blocks) and goes straight to selection.
 __device__ void select_row(float* s, int nb, float p, int k_min, int* __restrict__ out_idx,
                            int* __restrict__ out_cnt, unsigned long long* head_work,
-                           int* status, int lane) {
-  // softmax over the row, max subtracted
-  float m = -FLT_MAX;
-  for (int j = lane; j < nb; j += 32) m = fmaxf(m, s[j]);
-  m = warp_max(m);
-  float z = 0.f;
-  for (int j = lane; j < nb; j += 32) {
-    const float e = expf(s[j] - m);
-    s[j] = e;
-    z += e;
+                           int* status, int lane, bool softmax) {
+  if (softmax) {
+    // softmax over the row, max subtracted
+    float m = -FLT_MAX;
+    for (int j = lane; j < nb; j += 32) m = fmaxf(m, s[j]);
+    m = warp_max(m);
+    float z = 0.f;
+    for (int j = lane; j < nb; j += 32) {
+      const float e = expf(s[j] - m);
+      s[j] = e;
+      z += e;
+    }
+    z = warp_sum(z);
+    for (int j = lane; j < nb; j += 32) s[j] = s[j] / z;
+  } else {
+    // negative or non-finite importances are invalid input: clamped to 0, recorded
+    bool bad = false;
+    for (int j = lane; j < nb; j += 32) {
+      const float v = s[j];
+      if (!(v >= 0.f && v <= 1.f)) {
+        s[j] = v > 1.f ? 1.f : 0.f;
+        bad = true;
+      }
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) record_status(status, FVATTN_ERR_INVALID_ARG);
   }
-  z = warp_sum(z);
-  for (int j = lane; j < nb; j += 32) s[j] = s[j] / z;
   __syncwarp();
 
   int cnt;
@@ -240,7 +255,7 @@ __global__ void __launch_bounds__(kRouteThreads)
 __global__ void __launch_bounds__(kRouteThreads)
     select_rows_kernel(const float* __restrict__ S, int rows, int nb, float p, int k_min,
                        int* __restrict__ kv_idx, int* __restrict__ kv_cnt,
-                       unsigned long long* __restrict__ head_work, int* status) {
+                       unsigned long long* __restrict__ head_work, int* status, bool softmax) {
   extern __shared__ float4 smem_f4[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* srow = reinterpret_cast<float*>(smem_f4) + static_cast<size_t>(warp) * nb;
@@ -251,7 +266,7 @@ __global__ void __launch_bounds__(kRouteThreads)
   __syncwarp();
   const int bh = r / nb;
   select_row(srow, nb, p, k_min, kv_idx + static_cast<size_t>(r) * nb, kv_cnt + r, head_work + bh,
-             status, lane);
+             status, lane, softmax);
 }
 
 size_t route_scores_bytes(int BH, int nb) {
@@ -276,7 +291,22 @@ cudaError_t launch_route_select(const float* qbar, const float* kbar, float* S, 
   const int rows = BH * nb;
   const int warps = kRouteThreads / 32;
   select_rows_kernel<<<(rows + warps - 1) / warps, kRouteThreads, smem2, st>>>(
-      S, rows, nb, p, k_min, kv_idx, kv_cnt, head_work, status);
+      S, rows, nb, p, k_min, kv_idx, kv_cnt, head_work, status, true);
+  return cudaGetLastError();
+}
+
+// Top-p with the Top-k floor on given importance rows [BH, nb, nb] (no softmax).
+cudaError_t launch_select_topp(const float* rows_in, int BH, int nb, float p, int k_min, int* kv_idx,
+                               int* kv_cnt, unsigned long long* head_work, int* status,
+                               cudaStream_t st) {
+  const size_t smem = static_cast<size_t>(kRouteThreads / 32) * nb * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int rows = BH * nb;
+  const int warps = kRouteThreads / 32;
+  select_rows_kernel<<<(rows + warps - 1) / warps, kRouteThreads, smem, st>>>(
+      rows_in, rows, nb, p, k_min, kv_idx, kv_cnt, head_work, status, false);
   return cudaGetLastError();
 }
 

@@ -23,6 +23,8 @@
  * Diagnostic of mask quality, from statistics the attention kernels record:
  *   fvattn_block_importance  exact block importance   [GSRS §5.3, §A.2, §A.3]
  *   fvattn_attention_recall  attention recall of a mask            [GSRS §3.2]
+ *   fvattn_select_topp       Top-p + Top-k floor on exact importance: the
+ *                            GSRS search over a candidate set [GSRS §5.1, §5.2]
  * A second, static mask generator for the same attention kernel:
  *   fvattn_lvsa_lists  local window + rotating global frames        [LVSA §3]
  *
@@ -220,6 +222,24 @@ FVATTN_API fvattn_status fvattn_block_importance(const float* block_lse, const f
                                                  int B, int H, int N, int block,
                                                  float* importance, void* workspace,
                                                  size_t workspace_bytes, void* stream);
+
+/* Top-p selection with a Top-k floor on given importance rows [GSRS §5.1,
+ * §5.2, §5.3, §A.4]: the search step of GSRS, where the exact importance of a
+ * candidate set (fvattn_block_importance of a call over the candidate lists)
+ * chooses the blocks to keep. importance [B,H,nb,nb] fp32, each row
+ * non-negative and summing to one over its evaluated blocks (0 elsewhere).
+ * Per row, as in fvattn_route but without the softmax: n_p = the smallest c
+ * whose c largest importances sum to >= p (nb when p >= 1 or when no prefix
+ * reaches p), cnt = min(nb, max(n_p, k_min)), ties by lower block index; the
+ * selected blocks go to kv_idx [B,H,nb,nb] (ascending at [0, cnt)), kv_cnt
+ * [B,H,nb], head_work [B,H] = sum_i cnt. With p < 1 and k_min no larger than
+ * the candidate count, only candidates are selected. Entries outside [0, 1]
+ * are clamped and recorded as FVATTN_ERR_INVALID_ARG.
+ * Workspace: fvattn_workspace_bytes(FVATTN_OP_DIAG, ...). */
+FVATTN_API fvattn_status fvattn_select_topp(const float* importance, int B, int H, int N, int block,
+                                            float p, int k_min, int32_t* kv_idx, int32_t* kv_cnt,
+                                            int64_t* head_work, void* workspace,
+                                            size_t workspace_bytes, void* stream);
 
 /* Attention recall of a block mask [GSRS §3.2]: the fraction of the attention
  * weight that the listed blocks capture,

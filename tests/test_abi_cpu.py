@@ -257,3 +257,21 @@ def test_empty_inputs_are_rejected_before_any_launch():
     assert _lvsa(grid=g0) == F.FVATTN_ERR_INVALID_ARG
     assert _hilbert(grid=g0) == F.FVATTN_ERR_INVALID_ARG
     assert F.fvattn_workspace_bytes(F.FVATTN_OP_SPARSE_FWD, 1, 2, 0, 64, 64) == 0
+
+
+def _select(imp=FAKE, idx=FAKE, cnt=FAKE, hw=FAKE, p=0.8, k_min=1, B=1, H=2, N=256, block=64, ws=FAKE,
+            ws_bytes=256):
+    return F._lib.fvattn_select_topp(imp, B, H, N, block, p, k_min, idx, cnt, hw, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw, status", [
+    (dict(imp=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(hw=FAKE + 4), F.FVATTN_ERR_INVALID_ARG),
+    (dict(p=0.0), F.FVATTN_ERR_INVALID_ARG),
+    (dict(p=1.5), F.FVATTN_ERR_INVALID_ARG),
+    (dict(k_min=0), F.FVATTN_ERR_INVALID_ARG),
+    (dict(N=0), F.FVATTN_ERR_INVALID_ARG),
+    (dict(ws=None), F.FVATTN_ERR_WORKSPACE),
+])
+def test_select_topp_rejects(kw, status):
+    assert _select(**kw) == status

@@ -161,3 +161,59 @@ def test_importance_and_recall_sampled_480p():
         assert abs(rec[b, h, i] - float(O.attention_recall(ref, mask[b, h, i]))) <= RECALL_ABS
     print(f"wan1.3b-480p: mean recall of the routed mask {rec.mean():.4f}, "
           f"min {rec.min():.4f}, density {mask.mean():.3f}")
+
+
+def _select_gpu(w, imp_t, p, k_min):
+    dev = imp_t.device
+    nb = imp_t.shape[-1]
+    idx = torch.full((w.B, w.H, nb, nb), -1, dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.B, w.H, nb), dtype=torch.int32, device=dev)
+    hw = torch.empty((w.B, w.H), dtype=torch.int64, device=dev)
+    wsd = F.alloc_workspace(F.fvattn_workspace_bytes(F.FVATTN_OP_DIAG, w.B, w.H, w.N, w.d, w.block), dev)
+    F.fvattn_select_topp(imp_t, w.N, w.block, p, k_min, idx, cnt, hw, wsd)
+    assert F.fvattn_workspace_status(wsd) == F.FVATTN_OK
+    return idx.cpu().numpy(), cnt.cpu().numpy(), hw.cpu().numpy()
+
+
+@pytest.mark.parametrize("w", [ODD128, BS64], ids=lambda w: w.name)
+@pytest.mark.parametrize("p,k_min", [(0.8, 2), (0.5, 1), (1.0, 1)])
+def test_select_topp_on_importance_matches_oracle(w, p, k_min):
+    from parity import check_lists_valid, compare_masks
+    q, k, v = S.make_qkv(w, device="cuda")
+    grid, qp, kp, _, _, _ = _route_gpu(w, q, k)
+    vp = torch.empty_like(qp)
+    F.fvattn_permute(v, vp, grid)
+    _, _, imp = _diag_gpu(w, qp, kp, vp)                     # dense importance, fp32
+    idx, cnt, hw = _select_gpu(w, torch.from_numpy(imp).cuda(), p, k_min)
+    nb = grid.nb
+    check_lists_valid(idx, cnt, nb, k_min)
+    assert np.array_equal(hw, cnt.astype(np.int64).sum(-1))
+    scores = imp.astype(np.float64)
+    order = np.empty(scores.shape, dtype=np.int64)
+    ocnt = np.empty(scores.shape[:-1], dtype=np.int64)
+    for row in np.ndindex(*ocnt.shape):
+        order[row], ocnt[row] = O.topp_topk_select(scores[row], p, k_min)
+    n_mis, n_border, hard = compare_masks(mask_from_lists(idx, cnt, nb),
+                                          {"scores": scores, "order": order, "cnt": ocnt}, p)
+    assert not hard, hard[:3]
+    print(f"{w.name} p={p} k_min={k_min}: mismatched={n_mis} borderline={n_border}")
+
+
+def test_gsrs_search_over_candidates():
+    # candidates from the router, exact importance over them, then a tighter Top-p inside them
+    w = ODD128
+    q, k, v = S.make_qkv(w, device="cuda")
+    grid, qp, kp, kv_idx, kv_cnt, _ = _route_gpu(w, q, k)
+    vp = torch.empty_like(qp)
+    F.fvattn_permute(v, vp, grid)
+    _, _, imp = _diag_gpu(w, qp, kp, vp, kv_idx, kv_cnt)      # normalised over the candidates
+    nb = grid.nb
+    cand = mask_from_lists(kv_idx.cpu().numpy(), kv_cnt.cpu().numpy(), nb)
+    idx, cnt, _ = _select_gpu(w, torch.from_numpy(imp).cuda(), 0.8, 1)
+    sel = mask_from_lists(idx, cnt, nb)
+    assert np.all(sel <= cand)                                   # inside the candidate set
+    mass = np.where(sel, imp, 0.0).sum(-1)
+    assert np.all(mass >= 0.8 - 1e-5)                            # covers p of the candidates' mass
+    smallest = np.where(sel, imp, np.inf).min(-1)
+    assert np.all((cnt == 1) | (mass - smallest < 0.8 + 1e-5))   # minimal prefix
+    print(f"search: candidates density {cand.mean():.3f} -> {sel.mean():.3f}")
