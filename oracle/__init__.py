@@ -42,6 +42,14 @@ from .lvsa_oracle import (  # noqa: F401
     frame_mask,
     lvsa_block_mask,
 )
+from .lowprec_oracle import (  # noqa: F401
+    e4m3_encode,
+    e4m3_decode,
+    quantize_v,
+    dequantize_v,
+    masked_attention_qv,
+    masked_softmax_weights,
+)
 from .hilbert_oracle import (  # noqa: F401
     hilbert_index,
     hilbert_order,
