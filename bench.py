@@ -254,6 +254,39 @@ def run_lvsa(F, w, path, stream, warmup, eff_flops_fn):
             "head_work_max_over_mean": float(hwn.max() / hwn.mean()), "_lists": (idx, cnt)}
 
 
+def run_fp8v(F, w, path, stream, warmup, eff):
+    """Attention with the per-channel E4M3 V (8-bit P.V product) on the routed lists
+    of the timed call: the quantization step, the sparse and dense launches, and the
+    output's distance from the bf16-V launch on the same inputs."""
+    dev = path.qp.device
+    vq = torch.empty(path.vp.shape, dtype=torch.uint8, device=dev)
+    vs = torch.empty((w.B, w.H, w.d), dtype=torch.float32, device=dev)
+    wsq = F.alloc_workspace(F.fvattn_workspace_bytes(F.FVATTN_OP_QUANT_V, w.B, w.H, w.N, w.d, w.block), dev)
+    quant_ms = _median_ms(lambda: F.fvattn_quantize_v(path.vp, vq, vs, w.N, w.block, wsq), stream, warmup, 5)
+    out8 = torch.empty_like(path.op)
+    sparse_ms = _median_ms(lambda: F.fvattn_sparse_fwd_fp8v(path.qp, path.kp, vq, vs, out8, path.kv_idx,
+                                                            path.kv_cnt, w.N, w.block, path.ws_attn),
+                           stream, warmup, 3)
+    F.fvattn_sparse_fwd(path.qp, path.kp, path.vp, path.op, path.kv_idx, path.kv_cnt, w.N, w.block,
+                        path.ws_attn)
+    diff = (out8[:, :, :w.N].float() - path.op[:, :, :w.N].float()).abs()
+    dense_ms = _median_ms(lambda: F.fvattn_dense_fwd_fp8v(path.qp, path.kp, vq, vs, out8, w.N, w.block,
+                                                          path.ws_attn), stream, warmup, 3)
+    if F.fvattn_workspace_status(wsq) != F.FVATTN_OK or F.fvattn_workspace_status(path.ws_attn) != F.FVATTN_OK:
+        raise RuntimeError("kernel status word set in the FP8 V run")
+    v_bytes = w.B * w.H * w.N * w.d * 2
+    q_bytes = w.B * w.H * path.npad * w.d
+    d_flops = dense_flops(w.B, w.H, w.N, w.d)
+    return {"format": "E4M3, one fp32 scale per (b, h, channel); P rounded to E4M3 in the kernel",
+            "quantize_ms": quant_ms,
+            "quantize_gbs": (v_bytes + q_bytes) / (quant_ms * 1e-3) / 1e9,
+            "quantize_bytes": {"algorithmic": v_bytes + q_bytes, "moved": 2 * v_bytes + q_bytes,
+                               "note": "two passes over V: channel maxima, then encoding"},
+            "attention_ms": sparse_ms, "effective_tflops": eff / (sparse_ms * 1e-3) / 1e12,
+            "dense_attention_ms": dense_ms, "dense_tflops": d_flops / (dense_ms * 1e-3) / 1e12,
+            "max_abs_diff_vs_bf16_v": float(diff.max()), "mean_abs_diff_vs_bf16_v": float(diff.mean())}
+
+
 def run_hilbert(F, w, q, k, v, stream, warmup, eff_flops_fn):
     """The same call with blocks in Hilbert-curve order instead of 3-D tiles."""
     dev = q.device
@@ -426,6 +459,11 @@ def run_fvattn(args):
     if not args.no_diag:
         diag = run_diag(F, w, path, stream, args.warmup,
                         lvsa_lists=(lvsa.pop("_lists") if lvsa is not None else None))
+    fp8v = None
+    if not args.no_fp8v:
+        fp8v = run_fp8v(F, w, path, stream, args.warmup, eff)
+        fp8v["speedup_vs_bf16_v"] = ms_attn / fp8v["attention_ms"]
+        fp8v["dense_speedup_vs_bf16_v"] = ms_dense / fp8v["dense_attention_ms"]
 
     # ---- e2e through the public API with pinned host buffers: every step uploads its
     # q, k, v and downloads its output; HostPipeline overlaps the copies of
@@ -502,6 +540,16 @@ def run_fvattn(args):
         line["hilbert"] = hilbert
     if diag is not None:
         line["diag"] = diag
+    if fp8v is not None:
+        # Q.K^T stays bf16 and P.V runs on E4M3 at the nominal 2x rate: at equal halves of
+        # the FLOPs the tensor-core ceiling is 4/3 of the bf16 one.
+        a8 = eff / (fp8v["attention_ms"] * 1e-3) / 1e12
+        p8 = pk["bf16_sus"] * 4.0 / 3.0
+        fp8v["roofline"] = {"bound": "tensor", "kernel": "attn_fwd_sm100_kernel (E4M3 P.V)", "achieved": a8,
+                            "peak": p8, "unit": "TFLOP/s", "frac": a8 / p8,
+                            "peak_kind": f"{pk['source']} bf16 sustained x 4/3 (half the FLOPs at the "
+                                         f"nominal fp8/bf16 ratio of 2)"}
+        line["fp8v"] = fp8v
     if not args.no_cpu_baseline:
         tf, nblk, secs, cores = cpu_oracle_sample(w, q, k, v, path.kv_idx, path.kv_cnt,
                                                   budget_s=args.cpu_budget)
@@ -612,6 +660,7 @@ def main(argv=None):
     ap.add_argument("--no-diag", action="store_true", help="skip the GSRS block-importance diagnostic")
     ap.add_argument("--no-lvsa", action="store_true", help="skip the LVSA static-mask measurement")
     ap.add_argument("--no-hilbert", action="store_true", help="skip the Hilbert-order measurement")
+    ap.add_argument("--no-fp8v", action="store_true", help="skip the E4M3-V attention measurement")
     ap.add_argument("--sweep", action="store_true",
                     help="print the 720p p x k_min x block-size sweep (one JSON line per config) instead")
     ap.add_argument("--cpu-budget", type=float, default=15.0)

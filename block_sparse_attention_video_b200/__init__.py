@@ -9,7 +9,7 @@ fallback: importing it fails loudly if the library has not been built
 Entry points carry the C names: ``fvattn_permute``, ``fvattn_route``,
 ``fvattn_route_noalloc``, ``fvattn_sparse_fwd``, ``fvattn_dense_fwd``,
 ``fvattn_block_importance``, ``fvattn_attention_recall``, ``fvattn_select_topp``, ``fvattn_lvsa_lists``,
-``fvattn_hilbert_table``,
+``fvattn_hilbert_table``, ``fvattn_quantize_v``, ``fvattn_sparse_fwd_fp8v``, ``fvattn_dense_fwd_fp8v``,
 ``fvattn_workspace_bytes``, ``fvattn_workspace_status``. ``FVAttnPath`` strings them into the full per-call
 path (route -> permute V -> block-sparse attention -> inverse permute) over
 buffers it allocates once with torch; ``HostPipeline`` runs it over a sequence
@@ -51,13 +51,15 @@ FVATTN_OP_DENSE_FWD = 2
 FVATTN_OP_DIAG = 3
 FVATTN_OP_LVSA = 4
 FVATTN_OP_HILBERT = 5
+FVATTN_OP_QUANT_V = 6
 
 FVATTN_ORDER_TILES = 0
 FVATTN_ORDER_TABLE = 1
 
 EXPORTED = ("fvattn_workspace_bytes", "fvattn_permute", "fvattn_route", "fvattn_route_noalloc",
             "fvattn_sparse_fwd", "fvattn_dense_fwd", "fvattn_block_importance", "fvattn_attention_recall",
-            "fvattn_select_topp", "fvattn_lvsa_lists", "fvattn_hilbert_table",
+            "fvattn_select_topp", "fvattn_lvsa_lists", "fvattn_hilbert_table", "fvattn_quantize_v",
+            "fvattn_sparse_fwd_fp8v", "fvattn_dense_fwd_fp8v",
             "fvattn_workspace_status", "fvattn_status_string")
 
 
@@ -107,6 +109,15 @@ _lib.fvattn_dense_fwd.argtypes = [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c
                                   _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
                                   _c_void_p, _c_size_t, _c_void_p]
 _lib.fvattn_dense_fwd.restype = _c_int
+_lib.fvattn_quantize_v.argtypes = [_c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_void_p, _c_void_p,
+                                   _c_void_p, _c_size_t, _c_void_p]
+_lib.fvattn_quantize_v.restype = _c_int
+_lib.fvattn_sparse_fwd_fp8v.argtypes = [_c_void_p] * 9 + [_c_int] * 5 + [_c_float, _c_void_p, _c_size_t,
+                                                                      _c_void_p]
+_lib.fvattn_sparse_fwd_fp8v.restype = _c_int
+_lib.fvattn_dense_fwd_fp8v.argtypes = [_c_void_p] * 7 + [_c_int] * 5 + [_c_float, _c_void_p, _c_size_t,
+                                                                     _c_void_p]
+_lib.fvattn_dense_fwd_fp8v.restype = _c_int
 _lib.fvattn_block_importance.argtypes = [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int,
                                          _c_int, _c_int, _c_void_p, _c_void_p, _c_size_t, _c_void_p]
 _lib.fvattn_block_importance.restype = _c_int
@@ -233,6 +244,45 @@ def fvattn_dense_fwd(qp, kp, vp, out, N: int, block: int, workspace, scale=None,
     return out
 
 
+def fvattn_quantize_v(vp, vq, vscale, N: int, block: int, workspace, stream=None):
+    """Per-channel E4M3 quantization: vp [B,H,Npad,128] bf16 -> vq [B,H,Npad,128]
+    uint8 codes and vscale [B,H,128] fp32."""
+    _need_cuda(vp, vq, vscale, workspace)
+    B, H, _, d = vp.shape
+    if vp.dtype != torch.bfloat16 or vq.dtype != torch.uint8 or vscale.dtype != torch.float32:
+        raise TypeError("vp bf16, vq uint8, vscale float32")
+    _check(_lib.fvattn_quantize_v(_ptr(vp), B, H, N, d, block, _ptr(vq), _ptr(vscale), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream)),
+           "fvattn_quantize_v")
+    return vq, vscale
+
+
+def fvattn_sparse_fwd_fp8v(qp, kp, vq, vscale, out, kv_idx, kv_cnt, N: int, block: int, workspace,
+                           scale=None, lse=None, block_lse=None, stream=None):
+    """fvattn_sparse_fwd with the E4M3 V of fvattn_quantize_v (8-bit P.V product)."""
+    _need_cuda(qp, kp, vq, vscale, out, kv_idx, kv_cnt, workspace, lse, block_lse)
+    B, H, _, d = qp.shape
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(_lib.fvattn_sparse_fwd_fp8v(_ptr(qp), _ptr(kp), _ptr(vq), _ptr(vscale), _ptr(out), _ptr(lse),
+                                       _ptr(block_lse), _ptr(kv_idx), _ptr(kv_cnt), B, H, N, d, block, sc,
+                                       _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                       _stream(stream)), "fvattn_sparse_fwd_fp8v")
+    return out
+
+
+def fvattn_dense_fwd_fp8v(qp, kp, vq, vscale, out, N: int, block: int, workspace, scale=None, lse=None,
+                          block_lse=None, stream=None):
+    """fvattn_dense_fwd with the E4M3 V of fvattn_quantize_v (8-bit P.V product)."""
+    _need_cuda(qp, kp, vq, vscale, out, workspace, lse, block_lse)
+    B, H, _, d = qp.shape
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(_lib.fvattn_dense_fwd_fp8v(_ptr(qp), _ptr(kp), _ptr(vq), _ptr(vscale), _ptr(out), _ptr(lse),
+                                      _ptr(block_lse), B, H, N, d, block, sc, _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(stream)),
+           "fvattn_dense_fwd_fp8v")
+    return out
+
+
 def fvattn_block_importance(block_lse, lse, importance, N: int, block: int, workspace,
                             kv_idx=None, kv_cnt=None, stream=None):
     """Exact block importance [B,H,nb,nb] from an attention call's block_lse and lse
@@ -316,12 +366,17 @@ class FVAttnPath:
     also permutes q and k), permute v, block-sparse attention, inverse permute.
     ``dense=True`` runs the dense kernel instead of routing. ``order="hilbert"``
     orders blocks along the Hilbert curve (the table is built once here) instead
-    of 3-D tiles.
+    of 3-D tiles. ``v_format="e4m3"`` quantizes the permuted V per channel
+    (fvattn_quantize_v) and runs attention with the 8-bit P.V product.
     """
 
-    def __init__(self, B, H, grid, tile, block, d, dtype, p, k_min, device="cuda", order="tiles"):
+    def __init__(self, B, H, grid, tile, block, d, dtype, p, k_min, device="cuda", order="tiles",
+                 v_format="bf16"):
         if order not in ("tiles", "hilbert"):
             raise ValueError(f"unknown block order {order!r}")
+        if v_format not in ("bf16", "e4m3"):
+            raise ValueError(f"unknown V format {v_format!r}")
+        self.fp8v = v_format == "e4m3"
         table = fvattn_hilbert_table(grid, block, device) if order == "hilbert" else None
         self.grid = Grid.make(grid, tile, block, table=table)
         self.B, self.H, self.d = B, H, d
@@ -344,13 +399,26 @@ class FVAttnPath:
             fvattn_workspace_bytes(FVATTN_OP_ROUTE, B, H, self.N, d, block), dev)
         self.ws_attn = alloc_workspace(
             fvattn_workspace_bytes(FVATTN_OP_SPARSE_FWD, B, H, self.N, d, block), dev)
+        if self.fp8v:
+            self.vq = torch.empty(shp, dtype=torch.uint8, device=dev)
+            self.vscale = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+            self.ws_quant = alloc_workspace(
+                fvattn_workspace_bytes(FVATTN_OP_QUANT_V, B, H, self.N, d, block), dev)
 
     def route(self, q, k):
         fvattn_route(q, k, self.grid, self.p, self.k_min, self.kv_idx, self.kv_cnt,
                      self.head_work, self.ws_route, qp_out=self.qp, kp_out=self.kp)
 
     def attend(self, dense=False):
-        if dense:
+        if self.fp8v:
+            fvattn_quantize_v(self.vp, self.vq, self.vscale, self.N, self.block, self.ws_quant)
+            if dense:
+                fvattn_dense_fwd_fp8v(self.qp, self.kp, self.vq, self.vscale, self.op, self.N, self.block,
+                                      self.ws_attn)
+            else:
+                fvattn_sparse_fwd_fp8v(self.qp, self.kp, self.vq, self.vscale, self.op, self.kv_idx,
+                                       self.kv_cnt, self.N, self.block, self.ws_attn)
+        elif dense:
             fvattn_dense_fwd(self.qp, self.kp, self.vp, self.op, self.N, self.block, self.ws_attn)
         else:
             fvattn_sparse_fwd(self.qp, self.kp, self.vp, self.op, self.kv_idx, self.kv_cnt,

@@ -25,8 +25,8 @@ cudaError_t launch_attn_simt(const void* q, const void* k, const void* v, void* 
                              float* blse, const int* kv_idx, const int* kv_cnt, int BH, int N,
                              int d, int bs, bool bf16, float scale, int* status, cudaStream_t st);
 cudaError_t launch_attn_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                              void* out, float* lse, float* blse, const int* kv_idx,
-                              const int* kv_cnt,
+                              void* out, float* lse, float* blse, const float* vscale,
+                              const int* kv_idx, const int* kv_cnt,
                               uint32_t* ulist, int* ucnt, int* local_order,
                               unsigned long long* head_total, int* head_order, int BH, int N,
                               int nb, int bs, float scale, int* status,
@@ -41,6 +41,9 @@ cudaError_t launch_lvsa_lists(const TileGeom& g, int N, int bs, int window, int 
                               uint32_t* frames, cudaStream_t st);
 cudaError_t launch_hilbert_table(int T, int Hh, int W, int* table, unsigned long long* keys,
                                  cudaStream_t st);
+cudaError_t launch_quantize_v(const void* v, int BH, int N, int npad, uint8_t* vq, float* vscale,
+                              unsigned int* amax_bits, cudaStream_t st);
+size_t vquant_ws_bytes(int BH);
 int hilbert_bits(int extent);
 int next_pow2(int n);
 }  // namespace fvattn
@@ -146,6 +149,20 @@ bool make_row_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t bo
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [rows, 128] bytes (E4M3 V), row stride 128 B; box = box_rows rows x 128 bytes,
+// 128-byte swizzle.
+bool make_byte_row_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 fvattn_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA; }
 
 fvattn::TileGeom geom_of(const fvattn_grid* g) {
@@ -179,11 +196,15 @@ fvattn_status check_ws(const void* ws, size_t have, size_t need) {
 }
 
 // Common validation and dispatch of the attention forward (sparse or dense).
-fvattn_status attention_fwd(const void* qp, const void* kp, const void* vp, void* op, float* lse,
+// vscale != nullptr: vp holds E4M3 codes [B*H, Npad, 128] with per-channel
+// scales vscale [B*H, 128] (tensor-core path only).
+fvattn_status attention_fwd(const void* qp, const void* kp, const void* vp, const float* vscale,
+                            void* op, float* lse,
                             float* block_lse, const int32_t* kv_idx, const int32_t* kv_cnt, bool sparse, int B,
                             int H, int N, int d, fvattn_dtype dtype, int block, float scale,
                             void* ws, size_t ws_bytes, void* stream) {
   if (!qp || !kp || !vp || !op) return FVATTN_ERR_INVALID_ARG;
+  if (vscale && !aligned(vscale, 16)) return FVATTN_ERR_INVALID_ARG;
   if (!aligned(qp, 16) || !aligned(kp, 16) || !aligned(vp, 16) || !aligned(op, 16))
     return FVATTN_ERR_INVALID_ARG;
   if (lse && !aligned(lse, 4)) return FVATTN_ERR_INVALID_ARG;
@@ -192,6 +213,8 @@ fvattn_status attention_fwd(const void* qp, const void* kp, const void* vp, void
     return FVATTN_ERR_INVALID_ARG;
   if (!valid_dtype(dtype) || !valid_sizes(B, H, N, d, block)) return FVATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return FVATTN_ERR_INVALID_ARG;
+  const bool tensor_core = dtype == FVATTN_BF16 && d == 128;
+  if (vscale && !tensor_core) return FVATTN_ERR_UNSUPPORTED;
   const size_t need = fvattn_workspace_bytes(sparse ? FVATTN_OP_SPARSE_FWD : FVATTN_OP_DENSE_FWD,
                                              B, H, N, d, block);
   const fvattn_status wst = check_ws(ws, ws_bytes, need);
@@ -204,7 +227,6 @@ fvattn_status attention_fwd(const void* qp, const void* kp, const void* vp, void
   const int nb = num_blocks(N, block);
   if (cudaMemsetAsync(base, 0, kWsHeaderBytes, st) != cudaSuccess) return FVATTN_ERR_CUDA;
 
-  const bool tensor_core = dtype == FVATTN_BF16 && d == 128;
   if (!tensor_core) {
     return from_cuda(fvattn::launch_attn_simt(qp, kp, vp, op, lse, block_lse, sparse ? kv_idx : nullptr,
                                               sparse ? kv_cnt : nullptr, BH, N, d, block,
@@ -213,7 +235,7 @@ fvattn_status attention_fwd(const void* qp, const void* kp, const void* vp, void
   const uint64_t rows = static_cast<uint64_t>(BH) * nb * block;
   CUtensorMap tq, tk, tv;
   if (!make_row_map(&tq, qp, rows, 128) || !make_row_map(&tk, kp, rows, block) ||
-      !make_row_map(&tv, vp, rows, block))
+      !(vscale ? make_byte_row_map(&tv, vp, rows, block) : make_row_map(&tv, vp, rows, block)))
     return FVATTN_ERR_CUDA;
   const int sms = device_sm_count();
   if (sms <= 0) return FVATTN_ERR_CUDA;
@@ -231,7 +253,7 @@ fvattn_status attention_fwd(const void* qp, const void* kp, const void* vp, void
     head_order = reinterpret_cast<int*>(base + w.head_order);
   }
   return from_cuda(fvattn::launch_attn_sm100(
-      tq, tk, tv, op, lse, block_lse, sparse ? kv_idx : nullptr, sparse ? kv_cnt : nullptr, ulist, ucnt,
+      tq, tk, tv, op, lse, block_lse, vscale, sparse ? kv_idx : nullptr, sparse ? kv_cnt : nullptr, ulist, ucnt,
       local_order, head_total, head_order, BH, N, nb, block, scale, &hdr->status, &hdr->counter,
       sms, st));
 }
@@ -250,6 +272,8 @@ size_t fvattn_workspace_bytes(fvattn_op op, int B, int H, int N, int d, int bloc
     case FVATTN_OP_LVSA: return kWsHeaderBytes + align_up(num_blocks(N, block) * kLvsaBlockBytes, 256);
     case FVATTN_OP_HILBERT:
       return kWsHeaderBytes + align_up(static_cast<size_t>(fvattn::next_pow2(N)) * 8, 256);
+    case FVATTN_OP_QUANT_V:
+      return kWsHeaderBytes + align_up(fvattn::vquant_ws_bytes(B * H), 256);
   }
   return 0;
 }
@@ -315,7 +339,7 @@ fvattn_status fvattn_sparse_fwd(const void* qp, const void* kp, const void* vp, 
                                 const int32_t* kv_cnt, int B, int H, int N, int d,
                                 fvattn_dtype dtype, int block, float scale, void* workspace,
                                 size_t workspace_bytes, void* stream) {
-  return attention_fwd(qp, kp, vp, op, lse, block_lse, kv_idx, kv_cnt, true, B, H, N, d, dtype,
+  return attention_fwd(qp, kp, vp, nullptr, op, lse, block_lse, kv_idx, kv_cnt, true, B, H, N, d, dtype,
                        block, scale, workspace, workspace_bytes, stream);
 }
 
@@ -323,8 +347,51 @@ fvattn_status fvattn_dense_fwd(const void* qp, const void* kp, const void* vp, v
                                float* lse, float* block_lse, int B, int H, int N, int d,
                                fvattn_dtype dtype, int block, float scale, void* workspace,
                                size_t workspace_bytes, void* stream) {
-  return attention_fwd(qp, kp, vp, op, lse, block_lse, nullptr, nullptr, false, B, H, N, d,
+  return attention_fwd(qp, kp, vp, nullptr, op, lse, block_lse, nullptr, nullptr, false, B, H, N, d,
                        dtype, block, scale, workspace, workspace_bytes, stream);
+}
+
+fvattn_status fvattn_quantize_v(const void* vp, int B, int H, int N, int d, int block, uint8_t* vq,
+                                float* vscale, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  if (!vp || !vq || !vscale) return FVATTN_ERR_INVALID_ARG;
+  if (!aligned(vp, 16) || !aligned(vq, 16) || !aligned(vscale, 16)) return FVATTN_ERR_INVALID_ARG;
+  if (!valid_sizes(B, H, N, d, block)) return FVATTN_ERR_INVALID_ARG;
+  if (d != 128) return FVATTN_ERR_UNSUPPORTED;
+  const size_t npad = static_cast<size_t>(num_blocks(N, block)) * block;
+  const size_t bh = static_cast<size_t>(B) * H;
+  if (ranges_overlap(vp, bh * npad * d * 2, vq, bh * npad * d) ||
+      ranges_overlap(vp, bh * npad * d * 2, vscale, bh * d * 4) ||
+      ranges_overlap(vq, bh * npad * d, vscale, bh * d * 4))
+    return FVATTN_ERR_INVALID_ARG;
+  const size_t need = fvattn_workspace_bytes(FVATTN_OP_QUANT_V, B, H, N, d, block);
+  const fvattn_status wst = check_ws(workspace, workspace_bytes, need);
+  if (wst != FVATTN_OK) return wst;
+  auto st = static_cast<cudaStream_t>(stream);
+  auto base = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(base, 0, need, st) != cudaSuccess) return FVATTN_ERR_CUDA;
+  return from_cuda(fvattn::launch_quantize_v(vp, B * H, N, static_cast<int>(npad), vq, vscale,
+                                             reinterpret_cast<unsigned int*>(base + kWsHeaderBytes),
+                                             st));
+}
+
+fvattn_status fvattn_sparse_fwd_fp8v(const void* qp, const void* kp, const uint8_t* vq,
+                                     const float* vscale, void* op, float* lse, float* block_lse,
+                                     const int32_t* kv_idx, const int32_t* kv_cnt, int B, int H,
+                                     int N, int d, int block, float scale, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  if (!vscale) return FVATTN_ERR_INVALID_ARG;
+  return attention_fwd(qp, kp, vq, vscale, op, lse, block_lse, kv_idx, kv_cnt, true, B, H, N, d,
+                       FVATTN_BF16, block, scale, workspace, workspace_bytes, stream);
+}
+
+fvattn_status fvattn_dense_fwd_fp8v(const void* qp, const void* kp, const uint8_t* vq,
+                                    const float* vscale, void* op, float* lse, float* block_lse,
+                                    int B, int H, int N, int d, int block, float scale,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (!vscale) return FVATTN_ERR_INVALID_ARG;
+  return attention_fwd(qp, kp, vq, vscale, op, lse, block_lse, nullptr, nullptr, false, B, H, N, d,
+                       FVATTN_BF16, block, scale, workspace, workspace_bytes, stream);
 }
 
 fvattn_status fvattn_block_importance(const float* block_lse, const float* lse,

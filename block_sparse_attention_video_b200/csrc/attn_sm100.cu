@@ -49,6 +49,17 @@
 // Softmax: exponent base 2 with scale*log2(e) folded in, P rounded to bf16,
 // fp32 row sums. The running max is only raised (and O rescaled in TMEM) when a
 // block's max exceeds it by more than 8 (a factor 256), which keeps P <= 256.
+//
+// 8-bit V variant (F8 = true) [FVAttn §3.4: V is quantized on the GPU before
+// attention]: V arrives as E4M3 codes [B*H, Npad, 128] with one fp32 scale per
+// channel, and P.V runs as a kind::f8f6f4 MMA with P in E4M3 as well (P takes
+// 32 TMEM columns per 128 keys, four per 32-bit column; K = 32 per MMA). P is
+// formed relative to m_run - 4 with a rescale threshold of 4, so P <= 2^8 stays
+// inside E4M3's range (448) while values down to 2^-14 of 2^m_run keep a code.
+// The row sums add the E4M3 values actually multiplied (exact f16 pairs, summed
+// in f16 over 16 keys, then in fp32), so P/l stays a distribution. The channel
+// scales are applied with 1/l in the epilogue. A V stage is 16 KB: one
+// 128-byte swizzled row per key, read by an MN-major descriptor.
 #include <cfloat>
 
 #include "common.cuh"
@@ -65,7 +76,6 @@ constexpr int kRingBytes = 128 * 1024;
 constexpr int kThreads = 384;
 constexpr int kRegsSoftmax = 184;
 constexpr int kRegsControl = 128;
-constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.6931471805599453f;
 // One in kPolyEvery exponential pairs runs on the FMA pipe (exp2_poly3), the
 // rest on MUFU; 0 keeps every exponential on MUFU.
@@ -77,7 +87,7 @@ constexpr int kPolyEvery = FVATTN_POLY_EVERY;
 // A step covers 128 keys: one 128-token block, or two consecutive union entries
 // of 64-token blocks whose K (V) tiles are loaded into the two 64-row halves of
 // one 128-row stage. Every step is then an N = 128 S MMA and a K = 128 P.V.
-template <int BN>
+template <int BN, bool F8 = false>
 struct Tile {
   static constexpr int kStepKeys = 128;
   static constexpr int kBPS = kStepKeys / BN;              // union entries per step
@@ -87,7 +97,13 @@ struct Tile {
   static constexpr int kStages = kRingBytes / kKVBytes;
   static constexpr int kGroup = kUnitRows / BN;            // query blocks per unit
   static constexpr uint32_t kIdescQK = umma_idesc_bf16(128, kStepKeys, false);
-  static constexpr uint32_t kIdescPV = umma_idesc_bf16(128, HD, true);
+  static constexpr uint32_t kIdescPV =
+      F8 ? umma_idesc_e4m3(128, HD, true) : umma_idesc_bf16(128, HD, true);
+  static constexpr int kVBytes = F8 ? kStepKeys * HD : kKVBytes;    // V stage bytes
+  static constexpr int kPVK = F8 ? 32 : 16;                         // keys per P.V MMA
+  static constexpr int kPCols = kStepKeys / (F8 ? 4 : 2);           // TMEM columns of P
+  static constexpr float kPShift = F8 ? 4.0f : 0.0f;                // P relative to m_run - shift
+  static constexpr float kThreshold = F8 ? 4.0f : 8.0f;             // lazy rescale threshold
 };
 
 struct Params {
@@ -104,6 +120,7 @@ struct Params {
   __nv_bfloat16* out;
   float* lse;
   float* blse;              // nullable [B*H, nb, npad]: per (key block, row) log-sum-exp
+  const float* vscale;      // F8: [B*H, 128] per-channel scales of the E4M3 V
   int* status;
   unsigned long long* counter;
 };
@@ -173,12 +190,12 @@ __device__ __forceinline__ uint32_t entry_at(const Unit& x, int k, const Params&
   return e;
 }
 
-template <int BN>
+template <int BN, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const Params P) {
-  using T = Tile<BN>;
+  using T = Tile<BN, F8>;
   constexpr int kStages = T::kStages;
   extern __shared__ uint8_t smem_raw[];
   Smem<BN>& sm = *reinterpret_cast<Smem<BN>*>(
@@ -273,13 +290,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int t = 0; t < 2; ++t) {     // K(k) then V(k)
             const int s = it % kStages;
             if (!mbar_wait(&sm.kv_empty[s], ((it / kStages) & 1) ^ 1, abort_flag, P.status)) { ok = false; break; }
-            mbar_arrive_expect_tx(&sm.kv_full[s], T::kKVBytes);
             uint8_t* dst = sm.kv + s * T::kKVBytes;
-            const CUtensorMap* tm = t == 0 ? &tm_k : &tm_v;
+            if (F8 && t == 1) {
+              // E4M3 V: one 128-byte row (all channels) per key, one box per entry
+              mbar_arrive_expect_tx(&sm.kv_full[s], T::kVBytes);
 #pragma unroll
-            for (int h = 0; h < T::kBPS; ++h) {
-              tma_load_2d(dst + h * T::kSubBytes, tm, &sm.kv_full[s], 0, kvrow[h]);
-              tma_load_2d(dst + T::kKVHalf + h * T::kSubBytes, tm, &sm.kv_full[s], 64, kvrow[h]);
+              for (int h = 0; h < T::kBPS; ++h)
+                tma_load_2d(dst + h * T::kSubBytes, &tm_v, &sm.kv_full[s], 0, kvrow[h]);
+            } else {
+              mbar_arrive_expect_tx(&sm.kv_full[s], T::kKVBytes);
+              const CUtensorMap* tm = t == 0 ? &tm_k : &tm_v;
+#pragma unroll
+              for (int h = 0; h < T::kBPS; ++h) {
+                tma_load_2d(dst + h * T::kSubBytes, tm, &sm.kv_full[s], 0, kvrow[h]);
+                tma_load_2d(dst + T::kKVHalf + h * T::kSubBytes, tm, &sm.kv_full[s], 64, kvrow[h]);
+              }
             }
             ++it;
           }
@@ -336,11 +361,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int h = 0; h < 2; ++h) {
             if (!mbar_wait(&sm.p_full[X][h], pn[X] & 1, abort_flag, P.status)) return false;
             tc_fence_after();
+            constexpr int kPerHalf = T::kStepKeys / 2 / T::kPVK;
 #pragma unroll
-            for (int kk = h * (T::kStepKeys / 32); kk < (h + 1) * (T::kStepKeys / 32); ++kk) {
-              umma_ts(tmem + 256 + X * 128, tmem + X * 128 + kk * 8,
-                      umma_desc_sw128(va + kk * 2048, T::kKVHalf, 1024), T::kIdescPV,
-                      (k > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = h * kPerHalf; kk < (h + 1) * kPerHalf; ++kk) {
+              // kk-th K slice of P: 8 TMEM columns (16 bf16 or 32 E4M3 keys); of V:
+              // kPVK rows of 128 bytes
+              const uint64_t bd = umma_desc_sw128(va + kk * T::kPVK * 128, T::kKVHalf, 1024);
+              if constexpr (F8)
+                umma_ts_f8(tmem + 256 + X * 128, tmem + X * 128 + kk * 8, bd, T::kIdescPV,
+                           (k > 0 || kk > 0) ? 1u : 0u);
+              else
+                umma_ts(tmem + 256 + X * 128, tmem + X * 128 + kk * 8, bd, T::kIdescPV,
+                        (k > 0 || kk > 0) ? 1u : 0u);
             }
           }
           ++pn[X];
@@ -464,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // The decision is per row but tcgen05.ld/st are warp-collective: when
             // any row of the warp needs a larger max, the whole warp rescales,
             // rows that do not need it with factor 1.
-            const bool need = m_new > m_run + kRescaleThreshold;
+            const bool need = m_new > m_run + T::kThreshold;
             if (__any_sync(0xffffffffu, need)) {
               const float f = need ? ex2_approx(m_run - m_new) : 1.f;
               l_run *= f;
@@ -484,12 +516,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           // x = s * scale*log2(e) - m and the row sums in packed fp32x2 arithmetic.
           // Each half of P is published as soon as it is in TMEM.
           const float2 sl2x2 = make_float2(sl2, sl2);
-          const float2 negm = make_float2(-m_run, -m_run);
+          const float m_eff = m_run - T::kPShift;
+          const float2 negm = make_float2(-m_eff, -m_eff);
           float2 lc[NC];
 #pragma unroll
           for (int c = 0; c < NC; ++c) {
             uint32_t pk[16];
             float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            __half2 hs[2] = {__float2half2_rn(0.f), __float2half2_rn(0.f)};
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float2 xv = __ffma2_rn(
@@ -503,11 +537,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 p0 = ex2_approx(xv.x);
                 p1 = ex2_approx(xv.y);
               }
-              ls[i & 1] = __fadd2_rn(ls[i & 1], make_float2(p0, p1));
-              pk[i] = pack_bf16x2(p0, p1);
+              if constexpr (F8) {
+                // four keys per 32-bit word, lowest key in the low byte
+                const uint32_t q8 = pack_e4m3x2(p0, p1);
+                hs[i & 1] = __hadd2(hs[i & 1], e4m3x2_to_half2(q8));
+                pk[i >> 1] = (i & 1) ? (pk[i >> 1] | (q8 << 16)) : q8;
+              } else {
+                ls[i & 1] = __fadd2_rn(ls[i & 1], make_float2(p0, p1));
+                pk[i] = pack_bf16x2(p0, p1);
+              }
             }
-            lc[c] = __fadd2_rn(ls[0], ls[1]);
-            tmem_st16(tS + c * 16, pk);
+            if constexpr (F8) {
+              lc[c] = __half22float2(__hadd2(hs[0], hs[1]));
+              tmem_st8(tS + c * 8, reinterpret_cast<const uint32_t(&)[8]>(pk));
+            } else {
+              lc[c] = __fadd2_rn(ls[0], ls[1]);
+              tmem_st16(tS + c * 16, pk);
+            }
             if (c == NC / 2 - 1 || c == NC - 1) {
               tmem_wait_st();
               tc_fence_before();
@@ -526,14 +572,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             // sum, converted to the natural base.
             if (P.blse && mem[h] && qrow < P.npad)
               P.blse[(static_cast<size_t>(x.bh) * P.nb + (e[h] & 0xFFFFu)) * P.npad + qrow] =
-                  (m_run + __log2f(l_blk)) * kLn2;
+                  (m_eff + __log2f(l_blk)) * kLn2;
           }
         } else {
           uint32_t z[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) z[i] = 0u;
 #pragma unroll
-          for (int c = 0; c < NC; ++c) tmem_st16(tS + c * 16, z);
+          for (int c = 0; c < T::kPCols / 16; ++c) tmem_st16(tS + c * 16, z);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
@@ -552,6 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // warp-collective.
       const bool store = qrow < P.npad;
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      const float* vs = F8 ? P.vscale + static_cast<size_t>(x.bh) * HD : nullptr;
       const size_t grow = static_cast<size_t>(x.bh) * P.npad + qrow;
       uint4* orow = reinterpret_cast<uint4*>(P.out + grow * HD);
 #pragma unroll 1
@@ -560,16 +607,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tO + c * 32, o);
         tmem_wait_ld();
         uint32_t w[16];
+        if constexpr (F8) {
+          // O of the codes, times 1/l and each channel's scale
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+          for (int i = 0; i < 8; ++i) {
+            const float4 sc = __ldg(reinterpret_cast<const float4*>(vs + c * 32) + i);
+            w[2 * i] = pack_bf16x2(__uint_as_float(o[4 * i]) * (inv_l * sc.x),
+                                   __uint_as_float(o[4 * i + 1]) * (inv_l * sc.y));
+            w[2 * i + 1] = pack_bf16x2(__uint_as_float(o[4 * i + 2]) * (inv_l * sc.z),
+                                       __uint_as_float(o[4 * i + 3]) * (inv_l * sc.w));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+        }
         if (store) {
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             orow[c * 4 + i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
-      if (store && P.lse) P.lse[grow] = (m_run + __log2f(l_run)) * kLn2;
+      if (store && P.lse) P.lse[grow] = (m_run - T::kPShift + __log2f(l_run)) * kLn2;
       tc_fence_before();
     }
   }
@@ -716,22 +775,22 @@ __global__ void __launch_bounds__(1024)
 }
 
 // ---------------------------------------------------------------- launcher
-template <int BN>
+template <int BN, bool F8>
 static cudaError_t launch_bn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const sm100::Params& P, int num_sms, cudaStream_t st) {
   const size_t smem = sizeof(sm100::Smem<BN>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(sm100::attn_fwd_sm100_kernel<BN>,
+  cudaError_t e = cudaFuncSetAttribute(sm100::attn_fwd_sm100_kernel<BN, F8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int grid = max(1, min(num_sms, P.total_units));
-  sm100::attn_fwd_sm100_kernel<BN><<<grid, sm100::kThreads, smem, st>>>(tq, tk, tv, P);
+  sm100::attn_fwd_sm100_kernel<BN, F8><<<grid, sm100::kThreads, smem, st>>>(tq, tk, tv, P);
   return cudaGetLastError();
 }
 
 cudaError_t launch_attn_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                              void* out, float* lse, float* blse, const int* kv_idx,
-                              const int* kv_cnt,
+                              void* out, float* lse, float* blse, const float* vscale,
+                              const int* kv_idx, const int* kv_cnt,
                               uint32_t* ulist, int* ucnt, int* local_order,
                               unsigned long long* head_total, int* head_order, int BH, int N,
                               int nb, int bs, float scale, int* status,
@@ -763,9 +822,14 @@ cudaError_t launch_attn_sm100(const CUtensorMap& tq, const CUtensorMap& tk, cons
   P.out = static_cast<__nv_bfloat16*>(out);
   P.lse = lse;
   P.blse = blse;
+  P.vscale = vscale;
   P.status = status;
   P.counter = counter;
-  return bs == 64 ? launch_bn<64>(tq, tk, tv, P, num_sms, st) : launch_bn<128>(tq, tk, tv, P, num_sms, st);
+  if (vscale)
+    return bs == 64 ? launch_bn<64, true>(tq, tk, tv, P, num_sms, st)
+                    : launch_bn<128, true>(tq, tk, tv, P, num_sms, st);
+  return bs == 64 ? launch_bn<64, false>(tq, tk, tv, P, num_sms, st)
+                  : launch_bn<128, false>(tq, tk, tv, P, num_sms, st);
 }
 
 }  // namespace fvattn

@@ -104,7 +104,8 @@ typedef enum {
   FVATTN_OP_DENSE_FWD = 2,
   FVATTN_OP_DIAG = 3,     /* fvattn_block_importance, fvattn_attention_recall */
   FVATTN_OP_LVSA = 4,     /* fvattn_lvsa_lists */
-  FVATTN_OP_HILBERT = 5   /* fvattn_hilbert_table */
+  FVATTN_OP_HILBERT = 5,  /* fvattn_hilbert_table */
+  FVATTN_OP_QUANT_V = 6   /* fvattn_quantize_v */
 } fvattn_op;
 
 /* Workspace bytes needed by `op` for these sizes (0 if the sizes are invalid).
@@ -207,6 +208,47 @@ FVATTN_API fvattn_status fvattn_dense_fwd(const void* qp, const void* kp, const 
                                fvattn_dtype dtype, int block, float scale,
                                void* workspace, size_t workspace_bytes,
                                void* stream);
+
+/* Per-channel FP8 quantization of V [FVAttn §3.4: the GPU quantizes V in a
+ * step of its own before attention; the pages name no format].
+ * vp [B,H,Npad,128] bf16 in tile order (the input of fvattn_sparse_fwd);
+ * vq [B,H,Npad,128] uint8 E4M3 codes out (OCP FP8 E4M3: sign, 4 exponent bits
+ * with bias 7, 3 mantissa bits, largest finite 448); vscale [B,H,128] fp32 out.
+ * For each (b,h,channel c): amax_c = max |v| over the valid rows (< N);
+ *   vscale[c] = fp32(amax_c / 448) and
+ *   vq[r,c]   = round-to-nearest-even E4M3 of fp32(v[r,c] * fp32(448 / amax_c)),
+ * saturating at +-448 (both fp32 operations correctly rounded); a channel with
+ * amax_c < 2^-100 gets codes 0 and scale 0; rows >= N get code 0. The
+ * dequantized value is E4M3(vq) * vscale. d must be 128 (FVATTN_ERR_UNSUPPORTED
+ * otherwise); vp, vq and vscale 16-byte aligned and not overlapping.
+ * Workspace: fvattn_workspace_bytes(FVATTN_OP_QUANT_V, ...) (per-channel maxima). */
+FVATTN_API fvattn_status fvattn_quantize_v(const void* vp, int B, int H, int N, int d, int block,
+                                           uint8_t* vq, float* vscale, void* workspace,
+                                           size_t workspace_bytes, void* stream);
+
+/* Block-sparse attention forward with the FP8 V of fvattn_quantize_v:
+ * fvattn_sparse_fwd's definition with V replaced by E4M3(vq) * vscale. qp, kp
+ * bf16 [B,H,Npad,128]; vq, vscale as written by fvattn_quantize_v (16-byte
+ * aligned). Runs the tensor-core kernel with an 8-bit P.V product
+ * (kind::f8f6f4): P is rounded to E4M3 too, relative to a reference 2^4 below
+ * the running row max (so P <= 256 < 448), with row sums over the rounded P;
+ * the channel scales are applied with 1/l at the end. Q.K^T, the softmax
+ * statistics, lse and block_lse stay as in fvattn_sparse_fwd. d must be 128
+ * (FVATTN_ERR_UNSUPPORTED otherwise). Workspace: as fvattn_sparse_fwd. */
+FVATTN_API fvattn_status fvattn_sparse_fwd_fp8v(const void* qp, const void* kp, const uint8_t* vq,
+                                                const float* vscale, void* op, float* lse,
+                                                float* block_lse, const int32_t* kv_idx,
+                                                const int32_t* kv_cnt, int B, int H, int N, int d,
+                                                int block, float scale, void* workspace,
+                                                size_t workspace_bytes, void* stream);
+
+/* Dense attention forward with the FP8 V: fvattn_sparse_fwd_fp8v with every key
+ * block selected. Workspace: as fvattn_dense_fwd. */
+FVATTN_API fvattn_status fvattn_dense_fwd_fp8v(const void* qp, const void* kp, const uint8_t* vq,
+                                               const float* vscale, void* op, float* lse,
+                                               float* block_lse, int B, int H, int N, int d,
+                                               int block, float scale, void* workspace,
+                                               size_t workspace_bytes, void* stream);
 
 /* Exact block importance [GSRS §5.3, §A.2, §A.3] from the block_lse and lse
  * of one attention call (sparse or dense, same B, H, N, block):

@@ -275,3 +275,53 @@ def _select(imp=FAKE, idx=FAKE, cnt=FAKE, hw=FAKE, p=0.8, k_min=1, B=1, H=2, N=2
 ])
 def test_select_topp_rejects(kw, status):
     assert _select(**kw) == status
+
+
+def _quant(vp=FAKE, vq=FAKE + (1 << 24), vs=FAKE + (1 << 26), B=1, H=2, N=256, d=128, block=64, ws=FAKE + (1 << 28),
+           ws_bytes=1 << 20):
+    return F._lib.fvattn_quantize_v(vp, B, H, N, d, block, vq, vs, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw, status", [
+    (dict(vp=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(vq=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(vs=FAKE + (1 << 26) + 4), F.FVATTN_ERR_INVALID_ARG),
+    (dict(vq=FAKE + 4096), F.FVATTN_ERR_INVALID_ARG),            # overlaps vp
+    (dict(N=0), F.FVATTN_ERR_INVALID_ARG),
+    (dict(block=96), F.FVATTN_ERR_INVALID_ARG),
+    (dict(d=64), F.FVATTN_ERR_UNSUPPORTED),
+    (dict(ws=None), F.FVATTN_ERR_WORKSPACE),
+    (dict(ws_bytes=16), F.FVATTN_ERR_WORKSPACE),
+])
+def test_quantize_v_rejects(kw, status):
+    assert _quant(**kw) == status
+
+
+def test_quantize_v_workspace_holds_channel_maxima():
+    hdr = F.fvattn_workspace_bytes(F.FVATTN_OP_DENSE_FWD, 1, 1, 256, 128, 64)
+    assert F.fvattn_workspace_bytes(F.FVATTN_OP_QUANT_V, 2, 3, 256, 128, 64) >= hdr + 6 * 128 * 4
+
+
+def _fp8(sparse=True, vq=FAKE, vs=FAKE, d=128, idx=FAKE, scale=0.125, ws=FAKE, ws_bytes=1 << 30):
+    if sparse:
+        return F._lib.fvattn_sparse_fwd_fp8v(FAKE, FAKE, vq, vs, FAKE, None, None, idx, FAKE, 1, 2, 256, d, 64,
+                                             scale, ws, ws_bytes, None)
+    return F._lib.fvattn_dense_fwd_fp8v(FAKE, FAKE, vq, vs, FAKE, None, None, 1, 2, 256, d, 64, scale, ws,
+                                        ws_bytes, None)
+
+
+@pytest.mark.parametrize("sparse", [True, False])
+@pytest.mark.parametrize("kw, status", [
+    (dict(vs=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(vs=FAKE + 4), F.FVATTN_ERR_INVALID_ARG),
+    (dict(vq=None), F.FVATTN_ERR_INVALID_ARG),
+    (dict(scale=0.0), F.FVATTN_ERR_INVALID_ARG),
+    (dict(d=64), F.FVATTN_ERR_UNSUPPORTED),
+    (dict(ws=None), F.FVATTN_ERR_WORKSPACE),
+])
+def test_fp8v_attention_rejects(sparse, kw, status):
+    assert _fp8(sparse=sparse, **kw) == status
+
+
+def test_sparse_fp8v_rejects_missing_lists():
+    assert _fp8(idx=None) == F.FVATTN_ERR_INVALID_ARG
