@@ -47,7 +47,8 @@ METRIC = "sparse attn ms/call & effective TFLOP/s (Wan-14B 720p shape) vs own de
 # the kernel source they were taken on. They are reported only while the source
 # is unchanged; after any change the traffic is unknown and reported as null.
 ATTN_TRAFFIC = {
-    "wan14b-720p": {"bytes": 2.54e9 + 763.87e6, "src": "619c7d8a8f916bed"},
+    "wan14b-720p": {"bytes": 2.54e9 + 763.83e6, "src": "ca0b46e084ff1e5a"},
+    "wan14b-720p/fp8v": {"bytes": 2.01e9 + 760.17e6, "src": "ca0b46e084ff1e5a"},
 }
 ATTN_SRC = os.path.join(ROOT, "block_sparse_attention_video_b200", "csrc", "attn_sm100.cu")
 
@@ -547,6 +548,9 @@ def run_fvattn(args):
         p8 = pk["bf16_sus"] * 4.0 / 3.0
         fp8v["roofline"] = {"bound": "tensor", "kernel": "attn_fwd_sm100_kernel (E4M3 P.V)", "achieved": a8,
                             "peak": p8, "unit": "TFLOP/s", "frac": a8 / p8,
+                            "traffic": _attn_traffic(w.name + "/fp8v"),
+                            # Q, K read (2 B each), E4M3 V read (1 B), O written (2 B) per element
+                            "algorithmic_bytes": 7 * w.B * w.H * path.nb * w.block * w.d,
                             "peak_kind": f"{pk['source']} bf16 sustained x 4/3 (half the FLOPs at the "
                                          f"nominal fp8/bf16 ratio of 2)"}
         line["fp8v"] = fp8v
