@@ -47,8 +47,8 @@ METRIC = "sparse attn ms/call & effective TFLOP/s (Wan-14B 720p shape) vs own de
 # the kernel source they were taken on. They are reported only while the source
 # is unchanged; after any change the traffic is unknown and reported as null.
 ATTN_TRAFFIC = {
-    "wan14b-720p": {"bytes": 2.54e9 + 763.83e6, "src": "ca0b46e084ff1e5a"},
-    "wan14b-720p/fp8v": {"bytes": 2.01e9 + 760.17e6, "src": "ca0b46e084ff1e5a"},
+    "wan14b-720p": {"bytes": 2.55e9 + 764.74e6, "src": "7a980de0684eea7e"},
+    "wan14b-720p/fp8v": {"bytes": 2.02e9 + 758.44e6, "src": "7a980de0684eea7e"},
 }
 ATTN_SRC = os.path.join(ROOT, "block_sparse_attention_video_b200", "csrc", "attn_sm100.cu")
 
@@ -382,10 +382,19 @@ def replica_workload(w, rank: int):
     return w.replace(seed=w.seed + 1000 * rank)
 
 
+def _workload(args):
+    """The named workload; --block 64 runs it with 64-token blocks (1x8x8 tiles, as in the sweep)."""
+    w = S.WORKLOADS[args.workload]
+    if args.block and args.block != w.block:
+        w = w.replace(name=f"{w.name}-bs{args.block}", block=args.block,
+                      tile=(1, 8, 8) if args.block == 64 else (2, 8, 8))
+    return w
+
+
 def run_fvattn(args):
     import block_sparse_attention_video_b200 as F
     dist, rank, world, local = _dist_setup(args.gpus)
-    w = S.WORKLOADS[args.workload]
+    w = _workload(args)
     dev = torch.device("cuda", local)
     q, k, v = S.make_qkv(replica_workload(w, rank), device=dev)
     path = F.FVAttnPath(w.B, w.H, w.grid, w.tile, w.block, w.d, torch.bfloat16, w.p, w.k_min, device=dev)
@@ -573,7 +582,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     import oracle as O
-    w = S.WORKLOADS[args.workload]
+    w = _workload(args)
     cores = len(os.sched_getaffinity(0))
     q, k, v = S.make_qkv(w, device="cpu")
     perm = O.tile_order(*w.grid6)
@@ -659,6 +668,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("fvattn", "reference"), default="fvattn")
     ap.add_argument("--workload", default="wan14b-720p", choices=sorted(S.WORKLOADS))
+    ap.add_argument("--block", type=int, choices=(64, 128), default=None,
+                    help="run the workload with this block size (64: 1x8x8 tiles)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-diag", action="store_true", help="skip the GSRS block-importance diagnostic")

@@ -461,33 +461,73 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < NC; ++c) tmem_ld32(tS + c * 32, s[c]);
           tmem_wait_ld();
-          // Keys this row does not attend: the other half's block when the row's
-          // query block did not select it (or the pad half of an odd step), and
-          // the keys past N of the last block.
+          float mx = -FLT_MAX;
+          if constexpr (BPS == 1) {
+            // One block per step (the row attends it): only the keys past N of the
+            // last block are masked.
 #pragma unroll
-          for (int c = 0; c < NC; ++c) {
-            const int h = c / CPE;
-            const int kbase = (c % CPE) * 32;     // first key of the chunk within its block
-            if (!mem[h]) {
+            for (int c = 0; c < NC; ++c) {
+              const int kbase = c * 32;
+              if (static_cast<int>(e[0] & 0xFFFFu) == P.nb - 1 && tail < kbase + 32) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) s[c][i] = __float_as_uint(-INFINITY);
-            } else if (static_cast<int>(e[h] & 0xFFFFu) == P.nb - 1 && tail < kbase + 32) {
+                for (int i = 0; i < 32; ++i)
+                  if (kbase + i >= tail) s[c][i] = __float_as_uint(-INFINITY);
+              }
+            }
+            // Row max: 8 independent chains of 3-input max (exact in any order).
+            float mx8[8];
 #pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (kbase + i >= tail) s[c][i] = __float_as_uint(-INFINITY);
+            for (int i = 0; i < 8; ++i) mx8[i] = -FLT_MAX;
+#pragma unroll
+            for (int c = 0; c < NC; ++c)
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                mx8[i & 7] = fmax3(mx8[i & 7], __uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1]));
+            mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+          } else {
+            // Two 64-key entries per step. Keys this row does not attend:
+            //  * the half whose entry the row's query block did not select (or the
+            //    pad half of an odd step): it is left out of the row max below and
+            //    gets an exponent offset of -inf, so its P is exactly 0;
+            //  * the keys past N of the last block: set to -inf one by one. That is
+            //    rare and warp-uniform, so it sits behind a vote; written inline,
+            //    both maskings compile to selects over all 128 values on every step
+            //    (about half again the instructions of a one-block step).
+            bool tail_step = false;
+#pragma unroll
+            for (int h = 0; h < BPS; ++h)
+              tail_step |= mem[h] && static_cast<int>(e[h] & 0xFFFFu) == P.nb - 1 && tail < BN;
+            if (__any_sync(0xffffffffu, tail_step)) {
+#pragma unroll
+              for (int c = 0; c < NC; ++c) {
+                const int h = c / CPE;
+                const int kbase = (c % CPE) * 32;   // first key of the chunk within its block
+                const int v = static_cast<int>(e[h] & 0xFFFFu) == P.nb - 1 ? tail - kbase : 32;
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                  if (i >= v) s[c][i] = __float_as_uint(-INFINITY);
+              }
+            }
+            // Row max over the attended halves: per half, 8/BPS independent chains
+            // of 3-input max (exact in any order).
+            constexpr int kChains = 8 / BPS;
+#pragma unroll
+            for (int h = 0; h < BPS; ++h) {
+              float mc[kChains];
+#pragma unroll
+              for (int i = 0; i < kChains; ++i) mc[i] = -FLT_MAX;
+#pragma unroll
+              for (int c = h * CPE; c < (h + 1) * CPE; ++c)
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                  mc[i % kChains] = fmax3(mc[i % kChains], __uint_as_float(s[c][2 * i]),
+                                          __uint_as_float(s[c][2 * i + 1]));
+              float mh = mc[0];
+#pragma unroll
+              for (int i = 1; i < kChains; ++i) mh = fmaxf(mh, mc[i]);
+              if (mem[h]) mx = fmaxf(mx, mh);
             }
           }
-          // Row max: 8 independent chains of 3-input max (exact in any order).
-          float mx8[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) mx8[i] = -FLT_MAX;
-#pragma unroll
-          for (int c = 0; c < NC; ++c)
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              mx8[i & 7] = fmax3(mx8[i & 7], __uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1]));
-          const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                                 fmaxf(mx8[6], mx8[7]));
           const float m_new = mx * sl2;
           if (!have) {
             m_run = m_new;
@@ -523,11 +563,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < NC; ++c) {
             uint32_t pk[16];
             float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            // a half the row does not attend (two entries per step): every x = -inf, so P = 0
+            const float2 negc =
+                (BPS == 1 || mem[c / CPE]) ? negm : make_float2(-INFINITY, -INFINITY);
             __half2 hs[2] = {__float2half2_rn(0.f), __float2half2_rn(0.f)};
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float2 xv = __ffma2_rn(
-                  make_float2(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])), sl2x2, negm);
+                  make_float2(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])), sl2x2, negc);
               float p0, p1;
               if (kPolyEvery > 0 && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
                 const float2 pv = exp2_poly3x2(xv);
