@@ -217,6 +217,7 @@ def cpu_oracle_sample(w, q, k, v, kv_idx, kv_cnt, budget_s=15.0, seed=0):
 
 
 LVSA_WINDOW, LVSA_PERIOD, LVSA_STEP = 2, 8, 0
+GSRS_SEARCH_P = 0.9
 
 
 def _median_ms(fn, stream, warmup, reps):
@@ -349,10 +350,19 @@ def run_diag(F, w, path, stream, warmup, lvsa_lists=None):
     imp_ms = timed(lambda: F.fvattn_block_importance(blse, lse, imp, w.N, w.block, wsd,
                                                      kv_idx=path.kv_idx, kv_cnt=path.kv_cnt), 3)
     sparse_sum = float(imp.sum(-1).sub(1).abs().max())
+    # GSRS search step: Top-p (with the Top-k floor) on the exact importance of the
+    # routed candidates gives the next, smaller mask inside them.
+    idx2 = torch.empty_like(path.kv_idx)
+    cnt2 = torch.empty_like(path.kv_cnt)
+    hw2 = torch.empty_like(path.head_work)
+    select_ms = timed(lambda: F.fvattn_select_topp(imp, w.N, w.block, GSRS_SEARCH_P, w.k_min, idx2, cnt2, hw2,
+                                                   wsd), 3)
     F.fvattn_dense_fwd(path.qp, path.kp, path.vp, path.op, w.N, w.block, path.ws_attn, lse=lse,
                        block_lse=blse)
     F.fvattn_block_importance(blse, lse, imp, w.N, w.block, wsd)
     F.fvattn_attention_recall(imp, path.kv_idx, path.kv_cnt, rec, w.N, w.block, wsd)
+    rec2 = torch.empty_like(rec)
+    F.fvattn_attention_recall(imp, idx2, cnt2, rec2, w.N, w.block, wsd)
     rec_lvsa = None
     if lvsa_lists is not None:
         rec_lvsa = torch.empty_like(rec)
@@ -367,12 +377,17 @@ def run_diag(F, w, path, stream, warmup, lvsa_lists=None):
            "recall_of_routed_mask": {"mean": float(r.mean()), "p05": float(r.flatten().quantile(0.05)),
                                      "min": float(r.min())},
            "note": "GSRS block importance from block log-sum-exps; recall = dense importance captured by the "
-                   "routed lists"}
+                   "routed lists",
+           "search": {"p": GSRS_SEARCH_P, "k_min": w.k_min, "select_ms": select_ms,
+                      "density": float(cnt2.float().mean() / nb),
+                      "recall": {"mean": float(rec2.mean()), "p05": float(rec2.flatten().quantile(0.05)),
+                                 "min": float(rec2.min())},
+                      "note": "Top-p on the exact importance of the routed candidates (fvattn_select_topp)"}}
     if rec_lvsa is not None:
         rl = rec_lvsa.float()
         out["recall_of_lvsa_mask"] = {"mean": float(rl.mean()), "p05": float(rl.flatten().quantile(0.05)),
                                       "min": float(rl.min())}
-    del blse, imp
+    del blse, imp, idx2
     torch.cuda.empty_cache()
     return out
 
