@@ -260,3 +260,35 @@ def test_fp8v_path_sampled_720p():
     worst, rms, pred, gated = _check_fp8_rows(w, qn, kn, vh, mask[:, heads], outp, None, local)
     print(f"wan14b-720p fp8 V: {len(rows)} query blocks, max err {worst:.2e} rms {rms:.2e} "
           f"(predicted {pred:.2e}); rows gated {gated}")
+
+
+def test_fp8v_block_lse_gives_importance():
+    # block log-sum-exps of the E4M3 launch feed the GSRS importance: rows sum to one (block
+    # and row sums come from the same rounded P) and each entry stays within the P rounding
+    # of the exact importance. Each is a mean of ratios of sums of rounded P; with the
+    # relative rounding r = 2^-4 + N 2^-14 (normal steps, plus the subnormal steps of up to
+    # N keys against a row sum >= 1), a ratio is off by at most 2r / (1 - r) relative, plus
+    # the subnormal steps of one block, at most 128 * 2^-14 = 2^-7.
+    w = ODD128
+    q, k, _, vp, (qn, kn, _) = _inputs(w)
+    grid, qp, kp, kv_idx, kv_cnt, _ = _route_gpu(w, q, k)
+    vq, vs = _quant_gpu(w, vp)
+    nb = grid.nb
+    lse = torch.empty(qp.shape[:-1], dtype=torch.float32, device="cuda")
+    blse = torch.full((w.B, w.H, nb, qp.shape[2]), 12345.0, dtype=torch.float32, device="cuda")
+    op = torch.empty_like(qp)
+    ws = F.alloc_workspace(F.fvattn_workspace_bytes(F.FVATTN_OP_SPARSE_FWD, w.B, w.H, w.N, w.d, w.block), "cuda")
+    F.fvattn_sparse_fwd_fp8v(qp, kp, vq, vs, op, kv_idx, kv_cnt, w.N, w.block, ws, lse=lse, block_lse=blse)
+    assert F.fvattn_workspace_status(ws) == F.FVATTN_OK
+    imp = torch.empty((w.B, w.H, nb, nb), dtype=torch.float32, device="cuda")
+    wsd = F.alloc_workspace(F.fvattn_workspace_bytes(F.FVATTN_OP_DIAG, w.B, w.H, w.N, w.d, w.block), "cuda")
+    F.fvattn_block_importance(blse, lse, imp, w.N, w.block, wsd, kv_idx=kv_idx, kv_cnt=kv_cnt)
+    assert F.fvattn_workspace_status(wsd) == F.FVATTN_OK
+    got = imp.cpu().numpy()
+    mask = mask_from_lists(kv_idx.cpu().numpy(), kv_cnt.cpu().numpy(), nb)
+    ref = O.block_importance(qn, kn, mask, w.N, w.block, 1.0 / math.sqrt(w.d))
+    assert np.abs(got.sum(-1) - 1.0).max() <= 1e-4
+    assert np.all(got[~mask] == 0.0)
+    r = REL_P + w.N * SUB_P
+    assert np.all(np.abs(got - ref) <= 2 * r / (1 - r) * ref + 2.0 ** -7), np.abs(got - ref).max()
+    print(f"fp8 V importance: max |d| {np.abs(got - ref).max():.2e}, mean |d| {np.abs(got - ref)[mask].mean():.2e}")

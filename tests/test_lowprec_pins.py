@@ -189,3 +189,83 @@ def test_softmax_weights_rows_sum_to_one_and_reproduce_attention():
         assert np.allclose(w.sum(-1), 1.0)
         assert set(cols.tolist()) == set(range(0, 64)) | set(range(128, N))
         assert np.allclose(w @ v[cols], O.masked_attention_rows(q, k, v, mrow, N, bs, 0.3, i), atol=1e-12)
+
+
+# ---------------------------------------------------------------- planted mistakes
+# Modified copies of oracle steps; each must fail one of the checks that pin the oracle.
+
+def _encode_ties_away(x):
+    x = np.asarray(x, np.float64)
+    pos = Lp.e4m3_table()[:0x7F]
+    a = np.minimum(np.abs(x), 448.0)
+    hi = np.minimum(np.searchsorted(pos, a, side="left"), len(pos) - 1)
+    lo = np.maximum(hi - 1, 0)
+    pick_hi = (pos[hi] - a) <= (a - pos[lo])                # ties away from zero
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    return code | (np.signbit(x).astype(np.uint8) << 7)
+
+
+def _encode_truncating(x):
+    x = np.asarray(x, np.float64)
+    pos = Lp.e4m3_table()[:0x7F]
+    a = np.minimum(np.abs(x), 448.0)
+    code = (np.searchsorted(pos, a, side="right") - 1).astype(np.uint8)   # rounds toward zero
+    return code | (np.signbit(x).astype(np.uint8) << 7)
+
+
+def _quantize_amax_with_pad(v, N):
+    v32 = np.asarray(v, np.float32)
+    amax = np.abs(v32).max(axis=2)                            # pad rows counted
+    inv = (np.float32(448) / np.where(amax > 0, amax, 1)).astype(np.float32)
+    codes = Lp.e4m3_encode((v32 * inv[:, :, None, :]).astype(np.float32))
+    codes[:, :, N:, :] = 0
+    return codes, (amax / np.float32(448)).astype(np.float32)
+
+
+def _quantize_scale_inverted(v, N):
+    codes, scale = Lp.quantize_v(v, N)
+    return codes, np.where(scale > 0, np.float32(1) / np.where(scale > 0, scale, 1), 0).astype(np.float32)
+
+
+def _quantize_per_token(v, N):
+    v32 = np.asarray(v, np.float32)
+    amax = np.abs(v32).max(axis=3, keepdims=True)             # one scale per row, not per channel
+    inv = (np.float32(448) / np.where(amax > 0, amax, 1)).astype(np.float32)
+    codes = Lp.e4m3_encode((v32 * inv).astype(np.float32))
+    codes[:, :, N:, :] = 0
+    return codes, (amax[..., 0].max(axis=2) / np.float32(448)).astype(np.float32)
+
+
+def _encode_pin_holds(encode):
+    t = Lp.e4m3_table()[:0x7F]
+    mids = ((t[1:] + t[:-1]) / 2).astype(np.float32)
+    x = np.concatenate([mids, -mids, np.linspace(-460, 460, 4001, dtype=np.float32)])
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    return np.array_equal(encode(x), want)
+
+
+def _quantize_pins_hold(quantize):
+    v, codes, scale = _golden()
+    got_codes, got_scale = quantize(v[None, None], v.shape[0])
+    if not (np.array_equal(got_codes[0, 0], codes) and np.allclose(got_scale[0, 0], scale, rtol=1e-7, atol=0)):
+        return False
+    w = _v(N=300)
+    w[:, :, 300:] = 1e4
+    c1, s1 = quantize(w, 300)
+    c2, s2 = Lp.quantize_v(w, 300)
+    return np.array_equal(c1, c2) and np.array_equal(s1, s2)
+
+
+def test_pins_accept_the_oracle():
+    assert _encode_pin_holds(Lp.e4m3_encode)
+    assert _quantize_pins_hold(Lp.quantize_v)
+
+
+@pytest.mark.parametrize("bad", [_encode_ties_away, _encode_truncating])
+def test_planted_encoding_mistakes_are_caught(bad):
+    assert not _encode_pin_holds(bad)
+
+
+@pytest.mark.parametrize("bad", [_quantize_amax_with_pad, _quantize_scale_inverted, _quantize_per_token])
+def test_planted_quantization_mistakes_are_caught(bad):
+    assert not _quantize_pins_hold(bad)
