@@ -92,7 +92,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 2-D tiled bulk tensor load global -> shared (no multicast), completion via
+// 2-D tiled bulk tensor load global -> shared of this CTA only, completion via
 // the mbarrier's transaction count.
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map,
                                             uint64_t* bar, int x, int y) {
