@@ -219,7 +219,8 @@ FVATTN_API fvattn_status fvattn_dense_fwd(const void* qp, const void* kp, const 
  *   vq[r,c]   = round-to-nearest-even E4M3 of fp32(v[r,c] * fp32(448 / amax_c)),
  * saturating at +-448 (both fp32 operations correctly rounded); a channel with
  * amax_c < 2^-100 gets codes 0 and scale 0; rows >= N get code 0. The
- * dequantized value is E4M3(vq) * vscale. d must be 128 (FVATTN_ERR_UNSUPPORTED
+ * dequantized value is E4M3(vq) * vscale. V must be finite (a NaN is left out
+ * of amax_c and encodes as the NaN code). d must be 128 (FVATTN_ERR_UNSUPPORTED
  * otherwise); vp, vq and vscale 16-byte aligned and not overlapping.
  * Workspace: fvattn_workspace_bytes(FVATTN_OP_QUANT_V, ...) (per-channel maxima). */
 FVATTN_API fvattn_status fvattn_quantize_v(const void* vp, int B, int H, int N, int d, int block,
