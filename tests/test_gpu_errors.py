@@ -85,3 +85,38 @@ def test_invalid_lists_in_the_importance_kernels_are_reported():
     F.fvattn_attention_recall(imp, idx, cnt, rec, w.N, w.block, wsd)
     assert F.fvattn_workspace_status(wsd) == F.FVATTN_ERR_INVALID_ARG
     assert torch.isfinite(imp).all() and torch.isfinite(rec).all()
+
+
+def test_invalid_lists_in_the_fp8v_path_are_reported():
+    w = S.Workload("err-fp8v", 1, 2, 128, "bf16", (5, 12, 20), (1, 8, 8), 64, 0.9, 1, seed=65)
+    dev = torch.device("cuda")
+    q, k, v = S.make_qkv(w, device=dev)
+    grid = F.Grid.make(w.grid, w.tile, w.block)
+    nb = grid.nb
+    qp, kp, vp = (torch.empty((w.B, w.H, nb * w.block, w.d), dtype=q.dtype, device=dev) for _ in range(3))
+    for x, y in ((q, qp), (k, kp), (v, vp)):
+        F.fvattn_permute(x, y, grid)
+    vq = torch.empty(vp.shape, dtype=torch.uint8, device=dev)
+    vs = torch.empty((w.B, w.H, w.d), dtype=torch.float32, device=dev)
+    wsq = F.alloc_workspace(F.fvattn_workspace_bytes(F.FVATTN_OP_QUANT_V, w.B, w.H, w.N, w.d, w.block), dev)
+    F.fvattn_quantize_v(vp, vq, vs, w.N, w.block, wsq)
+    assert F.fvattn_workspace_status(wsq) == F.FVATTN_OK
+    idx, cnt = _lists(w, nb, dev)
+    good_idx, good_cnt = idx.clone(), cnt.clone()
+    cnt[0, 0, 1] = 0
+    idx[0, 1, 2, 1] = -3
+    op = torch.zeros_like(qp)
+    ws = F.alloc_workspace(F.fvattn_workspace_bytes(F.FVATTN_OP_SPARSE_FWD, w.B, w.H, w.N, w.d, w.block), dev)
+    F.fvattn_sparse_fwd_fp8v(qp, kp, vq, vs, op, idx, cnt, w.N, w.block, ws)
+    assert F.fvattn_workspace_status(ws) == F.FVATTN_ERR_INVALID_ARG
+    assert torch.isfinite(op[:, :, : w.N]).all()
+    # rows of untouched query blocks match a clean call up to rounding order (a broken
+    # list in the same 256-row unit changes how the unit's entries pair into steps)
+    op_good = torch.zeros_like(qp)
+    F.fvattn_sparse_fwd_fp8v(qp, kp, vq, vs, op_good, good_idx, good_cnt, w.N, w.block, ws)
+    assert F.fvattn_workspace_status(ws) == F.FVATTN_OK
+    bs = w.block
+    for (b, h, i) in [(0, 0, 0), (0, 1, 0), (0, 0, nb - 1)]:
+        rows = slice(i * bs, min((i + 1) * bs, w.N))
+        mx, _ = attention_errors(op[b, h, rows].float().cpu().numpy(), op_good[b, h, rows].float().cpu().numpy())
+        assert mx <= BF16_MAX_ABS, (b, h, i, mx)
