@@ -27,6 +27,12 @@
  *                            GSRS search over a candidate set [GSRS §5.1, §5.2]
  * A second, static mask generator for the same attention kernel:
  *   fvattn_lvsa_lists  local window + rotating global frames        [LVSA §3]
+ * Hilbert-curve block order, used through fvattn_grid.order:
+ *   fvattn_hilbert_table  the permutation table of a grid   [FVAttn §3.1; GSRS §A.6]
+ * Low-precision V [FVAttn §3.4]:
+ *   fvattn_quantize_v       per-channel E4M3 codes and scales of the permuted V
+ *   fvattn_sparse_fwd_fp8v, fvattn_dense_fwd_fp8v
+ *                           attention with that V (8-bit P.V on the tensor cores)
  *
  * Conventions (every entry point):
  *   - Tensors are dense, row-major, on the current CUDA device. A token row of
