@@ -1,6 +1,7 @@
 """GPU: HostPipeline (pinned host inputs and outputs, copies of neighbouring calls
 overlapping the current call's kernels) gives, call by call, exactly the output of
-FVAttnPath on device inputs (the kernels are deterministic per work unit)."""
+FVAttnPath on device inputs (the kernels are deterministic per work unit); a
+whole call captured in a CUDA graph (bf16 or E4M3 V) replays to the eager result."""
 
 import pytest
 import torch
@@ -36,11 +37,13 @@ def test_host_pipeline_matches_per_call_results(dense):
         assert torch.equal(host_out2[i], want[::-1][i].cpu()), i
 
 
+@pytest.mark.parametrize("v_format", ["bf16", "e4m3"])
 @pytest.mark.parametrize("dense", [False, True])
-def test_cuda_graph_replay_matches_eager(dense):
+def test_cuda_graph_replay_matches_eager(dense, v_format):
     w = S.WORKLOADS["wan1.3b-480p"]
     q, k, v = S.make_qkv(w, device="cuda")
-    path = F.FVAttnPath(w.B, w.H, w.grid, w.tile, w.block, w.d, torch.bfloat16, w.p, w.k_min)
+    path = F.FVAttnPath(w.B, w.H, w.grid, w.tile, w.block, w.d, torch.bfloat16, w.p, w.k_min,
+                        v_format=v_format)
     out = torch.empty_like(q)
     graph, res = path.capture_graph(q, k, v, dense=dense, out=out)
     for shift in (7, 19):
