@@ -239,9 +239,11 @@ FVATTN_API fvattn_status fvattn_quantize_v(const void* vp, int B, int H, int N, 
  * aligned). Runs the tensor-core kernel with an 8-bit P.V product
  * (kind::f8f6f4): P is rounded to E4M3 too, relative to a reference 2^4 below
  * the running row max (so P <= 256 < 448), with row sums over the rounded P;
- * the channel scales are applied with 1/l at the end. Q.K^T, the softmax
- * statistics, lse and block_lse stay as in fvattn_sparse_fwd. d must be 128
- * (FVATTN_ERR_UNSUPPORTED otherwise). Workspace: as fvattn_sparse_fwd. */
+ * the channel scales are applied with 1/l at the end. Q.K^T and the running
+ * max stay as in fvattn_sparse_fwd; lse and block_lse are formed from the row
+ * sums of the rounded P, so they carry its rounding (relative error of the sums
+ * at most about 2^-4). d must be 128 (FVATTN_ERR_UNSUPPORTED otherwise).
+ * Workspace: as fvattn_sparse_fwd. */
 FVATTN_API fvattn_status fvattn_sparse_fwd_fp8v(const void* qp, const void* kp, const uint8_t* vq,
                                                 const float* vscale, void* op, float* lse,
                                                 float* block_lse, const int32_t* kv_idx,
