@@ -371,14 +371,19 @@ class FVAttnPath:
     """
 
     def __init__(self, B, H, grid, tile, block, d, dtype, p, k_min, device="cuda", order="tiles",
-                 v_format="bf16"):
+                 v_format="bf16", _grid=None):
         if order not in ("tiles", "hilbert"):
             raise ValueError(f"unknown block order {order!r}")
         if v_format not in ("bf16", "e4m3"):
             raise ValueError(f"unknown V format {v_format!r}")
         self.fp8v = v_format == "e4m3"
-        table = fvattn_hilbert_table(grid, block, device) if order == "hilbert" else None
-        self.grid = Grid.make(grid, tile, block, table=table)
+        self._ctor = dict(grid=grid, tile=tile, block=block, d=d, dtype=dtype, p=p, k_min=k_min, device=device,
+                          order=order, v_format=v_format)
+        if _grid is not None:
+            self.grid = _grid                 # shared with the path it was split from
+        else:
+            table = fvattn_hilbert_table(grid, block, device) if order == "hilbert" else None
+            self.grid = Grid.make(grid, tile, block, table=table)
         self.B, self.H, self.d = B, H, d
         self.N, self.nb = self.grid.N, self.grid.nb
         self.npad = self.nb * block
@@ -404,6 +409,23 @@ class FVAttnPath:
             self.vscale = torch.empty((B, H, d), dtype=torch.float32, device=dev)
             self.ws_quant = alloc_workspace(
                 fvattn_workspace_bytes(FVATTN_OP_QUANT_V, B, H, self.N, d, block), dev)
+
+    def split_heads(self, groups):
+        """Paths over contiguous head ranges (B must be 1), each with its own buffers and
+        workspaces, sharing this path's grid (and Hilbert table). Heads are independent,
+        so running the sub-paths on head slices gives exactly this path's result.
+        Returns [(h0, h1, path)]."""
+        if self.B != 1:
+            raise ValueError("head groups need B == 1 (a head range is then contiguous)")
+        groups = max(1, min(int(groups), self.H))
+        bounds = [round(g * self.H / groups) for g in range(groups + 1)]
+        out = []
+        for h0, h1 in zip(bounds[:-1], bounds[1:]):
+            c = self._ctor
+            sub = FVAttnPath(1, h1 - h0, c["grid"], c["tile"], c["block"], c["d"], c["dtype"], self.p, self.k_min,
+                             device=c["device"], order=c["order"], v_format=c["v_format"], _grid=self.grid)
+            out.append((h0, h1, sub))
+        return out
 
     def route(self, q, k):
         fvattn_route(q, k, self.grid, self.p, self.k_min, self.kv_idx, self.kv_cnt,
@@ -466,62 +488,81 @@ class HostPipeline:
     neighbouring calls overlapping the kernels of the current one.
 
     Two device input sets and two output buffers alternate. Uploads run on one
-    copy stream, downloads on another, and the kernels on the current stream.
-    Events order them: call i's kernels wait for its upload; its download waits
-    for its kernels; the upload of call i+2 waits until call i's kernels have
-    read the shared input set; call i+2's kernels wait until call i's download
-    has read the shared output buffer.
+    copy stream, downloads on another. Events order them: call i's kernels wait
+    for its upload; its download waits for its kernels; the upload of call i+2
+    waits until call i's kernels have read the shared input set; call i+2's
+    kernels wait until call i's download has read the shared output buffer.
+
+    ``head_groups`` > 1 (B == 1) runs every call as that many head ranges, each on
+    its own stream with its own sub-path (FVAttnPath.split_heads), with the same
+    ordering per range. The heads are independent, so the results are the same;
+    the first range's kernels start after a fraction of the first upload, and the
+    last call's outputs start down as soon as each range is done.
     """
 
-    def __init__(self, path: FVAttnPath, dense=False):
+    def __init__(self, path: FVAttnPath, dense=False, head_groups=1):
         self.path = path
         self.dense = dense
         dev = path.qp.device
+        self.device = dev
         shp = (path.B, path.H, path.N, path.d)
         self.inp = [tuple(torch.empty(shp, dtype=path.dtype, device=dev) for _ in range(3)) for _ in range(2)]
         self.outp = [torch.empty(shp, dtype=path.dtype, device=dev) for _ in range(2)]
         self.up = torch.cuda.Stream(device=dev)
         self.down = torch.cuda.Stream(device=dev)
+        if head_groups > 1:
+            self.parts = path.split_heads(head_groups)
+            self.streams = [torch.cuda.Stream(device=dev) for _ in self.parts]
+        else:
+            self.parts = [(0, path.H, path)]
+            self.streams = [None]             # the caller's current stream
         self._ev = lambda: torch.cuda.Event()
-        self.done_read = [None, None]     # kernels of the last call on slot s have read its inputs
-        self.done_down = [None, None]     # download of the last call on slot s has read its output
+        g = len(self.parts)
+        self.done_read = [[None] * g for _ in range(2)]   # kernels of the last call on slot s read range g
+        self.done_down = [[None] * g for _ in range(2)]   # download of the last call on slot s read range g
 
     def run(self, host_qkv, host_out, start_event=None):
         """host_qkv: sequence of (q, k, v) pinned CPU tensors; host_out: sequence of
         pinned CPU tensors (may repeat). Enqueues every call; returns the event
         recorded on the current stream after the last download."""
-        comp = torch.cuda.current_stream(self.path.qp.device)
+        cur = torch.cuda.current_stream(self.device)
+        comps = [st if st is not None else cur for st in self.streams]
         if start_event is not None:
             self.up.wait_event(start_event)
             self.down.wait_event(start_event)
-        last = None
+        last = [None] * len(self.parts)
         for i, ((hq, hk, hv), ho) in enumerate(zip(host_qkv, host_out)):
             s = i & 1
             dq, dk, dv = self.inp[s]
-            with torch.cuda.stream(self.up):
-                if self.done_read[s] is not None:
-                    self.up.wait_event(self.done_read[s])
-                dq.copy_(hq, non_blocking=True)
-                dk.copy_(hk, non_blocking=True)
-                dv.copy_(hv, non_blocking=True)
-                ev_in = self._ev()
-                ev_in.record(self.up)
-            comp.wait_event(ev_in)
-            if self.done_down[s] is not None:
-                comp.wait_event(self.done_down[s])
-            self.path(dq, dk, dv, dense=self.dense, out=self.outp[s])
-            ev_k = self._ev()
-            ev_k.record(comp)
-            self.done_read[s] = ev_k
-            with torch.cuda.stream(self.down):
-                self.down.wait_event(ev_k)
-                ho.copy_(self.outp[s], non_blocking=True)
-                ev_d = self._ev()
-                ev_d.record(self.down)
-            self.done_down[s] = ev_d
-            last = ev_d
-        if last is not None:
-            comp.wait_event(last)
+            for g, (h0, h1, sub) in enumerate(self.parts):
+                hs = slice(h0, h1)
+                with torch.cuda.stream(self.up):
+                    if self.done_read[s][g] is not None:
+                        self.up.wait_event(self.done_read[s][g])
+                    dq[:, hs].copy_(hq[:, hs], non_blocking=True)
+                    dk[:, hs].copy_(hk[:, hs], non_blocking=True)
+                    dv[:, hs].copy_(hv[:, hs], non_blocking=True)
+                    ev_in = self._ev()
+                    ev_in.record(self.up)
+                comp = comps[g]
+                comp.wait_event(ev_in)
+                if self.done_down[s][g] is not None:
+                    comp.wait_event(self.done_down[s][g])
+                with torch.cuda.stream(comp):
+                    sub(dq[:, hs], dk[:, hs], dv[:, hs], dense=self.dense, out=self.outp[s][:, hs])
+                    ev_k = self._ev()
+                    ev_k.record(comp)
+                self.done_read[s][g] = ev_k
+                with torch.cuda.stream(self.down):
+                    self.down.wait_event(ev_k)
+                    ho[:, hs].copy_(self.outp[s][:, hs], non_blocking=True)
+                    ev_d = self._ev()
+                    ev_d.record(self.down)
+                self.done_down[s][g] = ev_d
+                last[g] = ev_d
+        for e in last:
+            if e is not None:
+                cur.wait_event(e)
         end = self._ev()
-        end.record(comp)
+        end.record(cur)
         return end

@@ -1,6 +1,7 @@
 """GPU: HostPipeline (pinned host inputs and outputs, copies of neighbouring calls
-overlapping the current call's kernels) gives, call by call, exactly the output of
-FVAttnPath on device inputs (the kernels are deterministic per work unit); a
+overlapping the current call's kernels, optionally per head range on separate
+streams) gives, call by call, exactly the output of FVAttnPath on device inputs
+(the kernels are deterministic per work unit); a
 whole call captured in a CUDA graph (bf16 or E4M3 V) replays to the eager result."""
 
 import pytest
@@ -14,18 +15,21 @@ if torch.cuda.is_available():
     import block_sparse_attention_video_b200 as F
 
 
+@pytest.mark.parametrize("head_groups", [1, 3])
 @pytest.mark.parametrize("dense", [False, True])
-def test_host_pipeline_matches_per_call_results(dense):
+def test_host_pipeline_matches_per_call_results(dense, head_groups):
     w = S.WORKLOADS["wan1.3b-480p"]
     calls = [S.make_qkv(w.replace(seed=w.seed + 100 * i), device="cuda") for i in range(3)]
     path = F.FVAttnPath(w.B, w.H, w.grid, w.tile, w.block, w.d, torch.bfloat16, w.p, w.k_min)
     want = [path(q, k, v, dense=dense).clone() for (q, k, v) in calls]
     host_in = [tuple(x.cpu().pin_memory() for x in qkv) for qkv in calls]
     host_out = [torch.empty(want[0].shape, dtype=want[0].dtype).pin_memory() for _ in calls]
-    pipe = F.HostPipeline(path, dense=dense)
+    pipe = F.HostPipeline(path, dense=dense, head_groups=head_groups)
     pipe.run(host_in, host_out)
     torch.cuda.synchronize()
-    assert F.fvattn_workspace_status(path.ws_attn) == F.FVATTN_OK
+    for _, _, sub in pipe.parts:
+        assert F.fvattn_workspace_status(sub.ws_attn) == F.FVATTN_OK
+        assert F.fvattn_workspace_status(sub.ws_route) == F.FVATTN_OK
     for i in range(len(calls)):
         assert torch.equal(host_out[i], want[i].cpu()), i
     # a second run reuses the same slots
