@@ -29,7 +29,8 @@ def test_host_pipeline_matches_per_call_results(dense, head_groups):
     torch.cuda.synchronize()
     for _, _, sub in pipe.parts:
         assert F.fvattn_workspace_status(sub.ws_attn) == F.FVATTN_OK
-        assert F.fvattn_workspace_status(sub.ws_route) == F.FVATTN_OK
+        if not dense:                     # a dense call does not route
+            assert F.fvattn_workspace_status(sub.ws_route) == F.FVATTN_OK
     for i in range(len(calls)):
         assert torch.equal(host_out[i], want[i].cpu()), i
     # a second run reuses the same slots
