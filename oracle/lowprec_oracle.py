@@ -40,7 +40,8 @@ AMAX_ZERO = 2.0 ** -100
 
 
 def e4m3_value(code: int) -> float:
-    """The real number an E4M3 byte encodes (NaN for the two NaN patterns)."""
+    """The real number an E4M3 byte encodes (NaN for the two NaN patterns).
+    [FVAttn §3.4] names no format; E4M3 is the reading (module header)."""
     s = (code >> 7) & 1
     e = (code >> 3) & 0xF
     m = code & 0x7
@@ -65,7 +66,8 @@ _POS = _TABLE[:E4M3_NAN_CODE]          # codes 0x00..0x7E, strictly increasing, 
 def e4m3_encode(x) -> np.ndarray:
     """Round each value to the nearest finite E4M3 number, ties to the even
     code (mantissa LSB 0), magnitudes above 448 to 448 (saturating). Returns the
-    codes as uint8; the sign bit follows the sign of x, zero included."""
+    codes as uint8; the sign bit follows the sign of x, zero included.
+    [FVAttn §3.4]; rounding rule: the reading in the module header."""
     x = np.asarray(x, np.float64)
     a = np.minimum(np.abs(x), E4M3_MAX)
     hi = np.searchsorted(_POS, a, side="left")          # _POS[hi-1] < a <= _POS[hi]
@@ -85,7 +87,9 @@ def e4m3_decode(codes) -> np.ndarray:
 
 def quantize_v(v, N: int):
     """Per-channel E4M3 quantization of V [B, H, Npad, d] (the bf16 values as
-    float32). Returns (codes uint8 [B, H, Npad, d], scale float32 [B, H, d])."""
+    float32). Returns (codes uint8 [B, H, Npad, d], scale float32 [B, H, d]).
+    [FVAttn §3.4: the GPU quantizes V before attention]; granularity and scale:
+    the reading in the module header."""
     v32 = np.asarray(v, np.float32)
     amax = np.abs(v32[:, :, :N, :]).max(axis=2)                      # exact
     nz = amax >= np.float32(AMAX_ZERO)
@@ -106,12 +110,13 @@ def dequantize_v(codes, scale) -> np.ndarray:
 def masked_attention_qv(qp, kp, codes, scale, mask, N: int, bs: int, sm_scale: float,
                         blocks=None) -> np.ndarray:
     """Block-sparse attention with the quantized V: the masked softmax over the
-    selected blocks' valid keys, times V^."""
+    selected blocks' valid keys, times V^. [FVAttn §2.1 (the masked attention),
+    §3.4 (V quantized)]"""
     return masked_attention(qp, kp, dequantize_v(codes, scale), mask, N, bs, sm_scale, blocks)
 
 
 def masked_softmax_weights(qp, kp, mask_row, N: int, bs: int, sm_scale: float, i: int):
-    """Softmax weights of the valid rows of query block ``i`` of one head over
+    """[FVAttn §2.1] Softmax weights of the valid rows of query block ``i`` of one head over
     the valid keys of its selected blocks. Returns (cols, w): the key positions
     and the fp64 weights [rows, len(cols)], each row summing to one."""
     qp = np.asarray(qp, np.float64)
