@@ -184,36 +184,74 @@ def _max_over_ranks(dist, v: float, device="cuda") -> float:
     return float(t.item())
 
 
-def cpu_oracle_sample(w, q, k, v, kv_idx, kv_cnt, budget_s=15.0, seed=0):
-    """Oracle masked attention on sampled query blocks of the GPU's mask; returns
-    (effective TFLOP/s, blocks, seconds, cores)."""
+def hbm_bytes(w, nb: int, cnt_sum: int) -> dict:
+    """Algorithmic HBM bytes of the bandwidth-bound kernels of one call.
+
+    route:   Q and K read in raster order (2 R), written in tile order with pad
+             rows (2 P), the fp32 block means (2 x nb x d x 4 per head) and the
+             selected list entries with their counts (4 B each);
+    permute: V read (R) and written in tile order (P);
+    inverse: the N valid output rows read and written back in raster order (2 R).
+    R = B*H*N*d*2 bytes, P = B*H*Npad*d*2 bytes (bf16)."""
+    bh = w.B * w.H
+    R = bh * w.N * w.d * 2
+    P = bh * nb * w.block * w.d * 2
+    route = 2 * R + 2 * P + 2 * bh * nb * w.d * 4 + 4 * cnt_sum + 4 * bh * nb
+    return {"route": route, "permute_v": R + P, "inverse": 2 * R}
+
+
+def _sample_query_blocks(rng, nb, cnt_row_max, per_head):
+    picks = set(rng.permutation(nb)[:per_head].tolist())
+    picks.add(nb - 1)                      # the ragged tail block
+    picks.add(int(cnt_row_max))            # the head's heaviest row
+    return sorted(picks)
+
+
+def oracle_check(w, qn, kn, vn, idx, cnt, op_perm, heads, per_head, rng, budget_s=None):
+    """The fp64 oracle on the host cores against one GPU call (test infrastructure:
+    runs only in the cpu_baseline leg and the sweep's parity check).
+
+    Routing of the given heads (permute, pool, scores, Top-p + floor) gives the
+    mask parity of the GPU's lists; masked attention of sampled query blocks of
+    those heads on the GPU's own mask gives the GPU output's error on those rows
+    (op_perm: the GPU output in tile order [B,H,Npad,d]). Returns (parity dict,
+    error dict, route seconds, attention seconds, attention FLOPs)."""
     import oracle as O
-    cores = len(os.sched_getaffinity(0))
-    perm = O.tile_order(*w.grid6)
+    from oracle.mask_parity import compare_masks, mask_from_lists, summary
     nb = w.nb
-    rng = np.random.default_rng(seed)
-    idx = kv_idx.cpu().numpy()
-    cnt = kv_cnt.cpu().numpy()
+    heads = list(heads)
+    t0 = time.perf_counter()
+    orc = O.route(qn[:, heads], kn[:, heads], w.grid6, w.block, w.p, w.k_min)
+    route_s = time.perf_counter() - t0
+    mask = mask_from_lists(idx[:, heads], cnt[:, heads], nb)
+    mp = summary(compare_masks(mask, orc, w.p))
+    mp["heads"] = len(heads)
+    perm = orc["perm"]
     n = np.full(nb, w.block, dtype=np.float64)
     n[-1] = w.N - (nb - 1) * w.block
     scale = 1.0 / math.sqrt(w.d)
-    flops = 0.0
-    blocks = 0
-    t0 = time.perf_counter()
-    heads = rng.permutation(w.H)
-    for h in heads:
-        qh, kh, vh = (O.permute(x[0, h].float().cpu().numpy().astype(np.float64), perm, w.block)
-                      for x in (q, k, v))
-        for i in rng.permutation(nb)[:4]:
-            mrow = np.zeros(nb, dtype=bool)
-            mrow[idx[0, h, i, :cnt[0, h, i]]] = True
-            O.masked_attention_rows(qh, kh, vh, mrow, w.N, w.block, scale, int(i))
-            flops += 4.0 * w.d * n[i] * n[mrow].sum()
+    flops, blocks, emax, esum, ecount = 0.0, 0, 0.0, 0.0, 0
+    t1 = time.perf_counter()
+    for hi, h in enumerate(heads):
+        qh, kh, vh = (O.permute(x[0, h].astype(np.float64), perm, w.block) for x in (qn, kn, vn))
+        for i in _sample_query_blocks(rng, nb, np.argmax(cnt[0, h]), per_head):
+            ref = O.masked_attention_rows(qh, kh, vh, mask[0, hi, i], w.N, w.block, scale, int(i))
+            got = op_perm[0, h, i * w.block:i * w.block + ref.shape[0]].astype(np.float64)
+            e = np.abs(got - ref)
+            emax = max(emax, float(e.max()))
+            esum += float(e.sum())
+            ecount += e.size
+            flops += 4.0 * w.d * n[i] * n[mask[0, hi, i]].sum()
             blocks += 1
-        if time.perf_counter() - t0 > budget_s:
+        if budget_s is not None and time.perf_counter() - t1 > budget_s:
             break
-    dt = time.perf_counter() - t0
-    return flops / dt / 1e12, blocks, dt, cores
+    attn_s = time.perf_counter() - t1
+    mean = esum / max(1, ecount)
+    err = {"query_blocks": blocks, "max_abs": emax, "mean_abs": mean,
+           "tolerance": {"max_abs": 2e-2, "mean_abs": 2e-3},
+           "within_tolerance": bool(emax <= 2e-2 and mean <= 2e-3),
+           "against": "fp64 oracle masked attention on the GPU's own mask"}
+    return mp, err, route_s, attn_s, flops, blocks
 
 
 LVSA_WINDOW, LVSA_PERIOD, LVSA_STEP = 2, 8, 0
@@ -416,15 +454,22 @@ def run_fvattn(args):
     path = F.FVAttnPath(w.B, w.H, w.grid, w.tile, w.block, w.d, torch.bfloat16, w.p, w.k_min, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(ev_attn=None):
+    def step(ev=None):
+        # ev: five events around the four calls (route, V permute, attention, inverse)
+        if ev is not None:
+            ev[0].record(stream)
         path.route(q, k)
+        if ev is not None:
+            ev[1].record(stream)
         F.fvattn_permute(v, path.vp, path.grid)
-        if ev_attn is not None:
-            ev_attn[0].record(stream)
+        if ev is not None:
+            ev[2].record(stream)
         path.attend()
-        if ev_attn is not None:
-            ev_attn[1].record(stream)
+        if ev is not None:
+            ev[3].record(stream)
         F.fvattn_permute(path.op, path.out, path.grid, inverse=True)
+        if ev is not None:
+            ev[4].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -438,8 +483,8 @@ def run_fvattn(args):
     hw = path.head_work.cpu().numpy().astype(np.float64)
     work_ratio = float(hw.max() / hw.mean())
 
-    # ---- timed region: K full steps, per-launch events around the attention kernel
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # ---- timed region: K full steps, events around each call of a step
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(5)) for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
         if os.environ.get("CUDA_VISIBLE_DEVICES") else local
@@ -454,8 +499,11 @@ def run_fvattn(args):
         _barrier(dist)
     clocks = clk.summary()
     ms_step = start.elapsed_time(end) / args.steps
-    attn_ms = [a.elapsed_time(b) for a, b in ev]
-    ms_attn = sum(attn_ms) / len(attn_ms)
+
+    def call_ms(i):
+        return sum(e[i].elapsed_time(e[i + 1]) for e in ev) / len(ev)
+
+    ms_route, ms_vperm, ms_attn, ms_inv = (call_ms(i) for i in range(4))
     ms_step_max = _max_over_ranks(dist, ms_step)
     launches_per_step = 9   # gather_pool, block scores, select rows, permute V, plan x3, attention, inverse
 
@@ -531,6 +579,9 @@ def run_fvattn(args):
 
     pk = _peaks()
     achieved = eff / (ms_attn * 1e-3) / 1e12
+    hb = hbm_bytes(w, path.nb, int(cnt_np.astype(np.int64).sum()))
+    hbm_ms = ms_route + ms_vperm + ms_inv
+    hbm_achieved = (hb["route"] + hb["permute_v"] + hb["inverse"]) / (hbm_ms * 1e-3) / 1e9
     line = {
         "metric": METRIC,
         "value": world * eff / (ms_step_max * 1e-3) / 1e12,
@@ -539,12 +590,10 @@ def run_fvattn(args):
         "ms_per_step": ms_step_max,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "grid": list(w.grid),
-                   "tiles": list(w.tile), "block": w.block, "p": w.p, "k_min": w.k_min,
-                   "l2": f"inputs larger than L2 (Q, K, V {w.B * w.H * w.N * w.d * 2 / 1e6:.0f} MB each); "
-                         f"no flush",
-                   "parallelism": f"independent replicas x{world}"},
+        "config": bench_config(w, world),
         "ms_per_call": ms_step_max,
+        "ms_per_call_by_step": {"route": ms_route, "permute_v": ms_vperm, "attention": ms_attn,
+                                "inverse_permute": ms_inv},
         "attention_ms_per_launch": ms_attn,
         "effective_tflop_per_call": eff / 1e12,
         "density": density,
@@ -558,6 +607,13 @@ def run_fvattn(args):
                      "frac_of_burst_peak": achieved / pk["bf16"],
                      "traffic": _attn_traffic(w.name), "traffic_unit": "bytes per launch (DRAM read + write)",
                      "algorithmic_bytes": 4 * w.B * w.H * path.nb * w.block * w.d * 2},
+        "roofline_hbm": {"bound": "hbm", "kernels": "route (gather + pool, block scores, select) + V permute + "
+                                                    "inverse permute",
+                         "achieved": hbm_achieved, "peak": pk["hbm"], "unit": "GB/s",
+                         "frac": hbm_achieved / pk["hbm"], "peak_kind": f"{pk['source']} HBM copy bandwidth",
+                         "ms": hbm_ms, "algorithmic_bytes": hb,
+                         "traffic": None,
+                         "note": "CUDA events around each call inside the timed steps; bytes as in hbm_bytes()"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
@@ -584,16 +640,48 @@ def run_fvattn(args):
                                          f"nominal fp8/bf16 ratio of 2)"}
         line["fp8v"] = fp8v
     if not args.no_cpu_baseline:
-        tf, nblk, secs, cores = cpu_oracle_sample(w, q, k, v, path.kv_idx, path.kv_cnt,
-                                                  budget_s=args.cpu_budget)
-        line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                                "sample": f"fp64 oracle block-sparse attention of {nblk} query blocks "
-                                          f"(4 per head, random heads) of this call on the GPU's mask, "
-                                          f"{secs:.1f} s"}
+        # The timed call once more (the diagnostics above overwrite the output
+        # buffer), then the oracle on the host cores: routing of every head for the
+        # mask parity, masked attention of sampled query blocks for the output error
+        # and the oracle's throughput.
+        step()
+        torch.cuda.synchronize()
+        idx2, cnt2 = path.kv_idx.cpu().numpy(), path.kv_cnt.cpu().numpy()
+        same_lists = bool(np.array_equal(cnt2, cnt_np) and all(
+            np.array_equal(idx2[r][:c], idx_np[r][:c]) for r, c in np.ndenumerate(cnt_np)))
+        cores = len(os.sched_getaffinity(0))
+        qn, kn, vn = (x.float().cpu().numpy() for x in (q, k, v))
+        op_perm = path.op.float().cpu().numpy()
+        rng = np.random.default_rng(0)
+        mp, err, route_s, attn_s, oflops, nblk = oracle_check(
+            w, qn, kn, vn, idx2, cnt2, op_perm, range(w.H), per_head=2, rng=rng, budget_s=args.cpu_budget)
+        mp["lists_identical_across_calls"] = same_lists
+        del qn, kn, vn, op_perm
+        tf = oflops / attn_s / 1e12
+        line["mask_parity"] = mp
+        line["output_error"] = err
+        line["cpu_baseline"] = {
+            "value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 oracle block-sparse attention of {nblk} query blocks of this call (the tail "
+                      f"block, each head's heaviest row and random ones) on the GPU's mask, {attn_s:.1f} s; "
+                      f"routing of all {w.H} heads {route_s:.1f} s",
+            "oracle_ms_per_query_block": attn_s * 1e3 / max(1, nblk),
+            "oracle_route_ms": route_s * 1e3,
+            "extrapolated_call_ms": route_s * 1e3 + eff / (tf * 1e12) * 1e3,
+            "extrapolated_note": "EXTRAPOLATED: measured routing of every head plus this call's effective "
+                                 "FLOPs at the sampled blocks' oracle throughput"}
     print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()
     return 0
+
+
+def bench_config(w, world: int) -> dict:
+    """The config dict of the JSON line (the same for both arms)."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "grid": list(w.grid),
+            "tiles": list(w.tile), "block": w.block, "p": w.p, "k_min": w.k_min,
+            "l2": f"inputs larger than L2 (Q, K, V {w.B * w.H * w.N * w.d * 2 / 1e6:.0f} MB each); no flush",
+            "parallelism": f"independent replicas x{world}"}
 
 
 def run_reference(args):
@@ -639,8 +727,7 @@ def run_reference(args):
             "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "block": w.block,
-                       "p": w.p, "k_min": w.k_min},
+            "config": bench_config(w, int(os.environ.get("WORLD_SIZE", "1"))),
             "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": "per step: one head's fp64 routing (permute, pool, scores, "
                                        "Top-p) and block-sparse attention of 2 query blocks"},
@@ -649,14 +736,21 @@ def run_reference(args):
     return 0
 
 
+SWEEP_PARITY_HEADS = range(0, 40, 5)
+
+
 def run_sweep(args):
     """The 720p sweep (p x k_min x block size): one JSON line per config with its
-    density, route and attention times and effective TFLOP/s (not the headline line)."""
+    density, route and attention times and effective TFLOP/s (not the headline line),
+    and, unless --no-cpu-baseline, its parity against the fp64 oracle: the masks of
+    every query block of 8 heads (every fifth) and the outputs of each such head's
+    tail block and heaviest row."""
     import block_sparse_attention_video_b200 as F
     _dist_setup(1)
     base = S.WORKLOADS["wan14b-720p"]
     q, k, v = S.make_qkv(base, device="cuda")
     stream = torch.cuda.current_stream()
+    host = None if args.no_cpu_baseline else tuple(x.float().cpu().numpy() for x in (q, k, v))
     paths = {}
     for w in S.sweep_workloads():
         key = (w.block, w.tile)
@@ -674,10 +768,16 @@ def run_sweep(args):
         idx, cnt = path.kv_idx.cpu().numpy(), path.kv_cnt.cpu().numpy()
         eff = effective_flops(idx, cnt, w.N, w.block, w.d)
         hw = path.head_work.cpu().numpy().astype(np.float64)
-        print(json.dumps({"sweep": w.name, "block": w.block, "p": w.p, "k_min": w.k_min,
-                          "density": float(cnt.mean() / path.nb), "route_ms": route_ms, "attention_ms": attn_ms,
-                          "effective_tflops": eff / (attn_ms * 1e-3) / 1e12,
-                          "head_work_max_over_mean": float(hw.max() / hw.mean())}), flush=True)
+        rec = {"sweep": w.name, "block": w.block, "p": w.p, "k_min": w.k_min,
+               "density": float(cnt.mean() / path.nb), "route_ms": route_ms, "attention_ms": attn_ms,
+               "effective_tflops": eff / (attn_ms * 1e-3) / 1e12,
+               "head_work_max_over_mean": float(hw.max() / hw.mean())}
+        if host is not None:
+            mp, err, _, _, _, _ = oracle_check(w, *host, idx, cnt, path.op.float().cpu().numpy(),
+                                               SWEEP_PARITY_HEADS, per_head=0, rng=np.random.default_rng(0))
+            rec["mask_parity"] = mp
+            rec["output_error"] = err
+        print(json.dumps(rec), flush=True)
     return 0
 
 

@@ -10,7 +10,8 @@ Entry points carry the C names: ``fvattn_permute``, ``fvattn_route``,
 ``fvattn_route_noalloc``, ``fvattn_sparse_fwd``, ``fvattn_dense_fwd``,
 ``fvattn_block_importance``, ``fvattn_attention_recall``, ``fvattn_select_topp``, ``fvattn_lvsa_lists``,
 ``fvattn_hilbert_table``, ``fvattn_quantize_v``, ``fvattn_sparse_fwd_fp8v``, ``fvattn_dense_fwd_fp8v``,
-``fvattn_workspace_bytes``, ``fvattn_workspace_status``. ``FVAttnPath`` strings them into the full per-call
+``fvattn_workspace_bytes``, ``fvattn_workspace_status``, ``fvattn_wait_selftest``. ``FVAttnPath`` strings
+them into the full per-call
 path (route -> permute V -> block-sparse attention -> inverse permute) over
 buffers it allocates once with torch; ``HostPipeline`` runs it over a sequence
 of calls with pinned host inputs and outputs, overlapping the copies of
@@ -60,7 +61,7 @@ EXPORTED = ("fvattn_workspace_bytes", "fvattn_permute", "fvattn_route", "fvattn_
             "fvattn_sparse_fwd", "fvattn_dense_fwd", "fvattn_block_importance", "fvattn_attention_recall",
             "fvattn_select_topp", "fvattn_lvsa_lists", "fvattn_hilbert_table", "fvattn_quantize_v",
             "fvattn_sparse_fwd_fp8v", "fvattn_dense_fwd_fp8v",
-            "fvattn_workspace_status", "fvattn_status_string")
+            "fvattn_workspace_status", "fvattn_status_string", "fvattn_wait_selftest")
 
 
 class Grid(ctypes.Structure):
@@ -134,6 +135,8 @@ _lib.fvattn_hilbert_table.argtypes = [ctypes.POINTER(Grid), _c_void_p, _c_void_p
 _lib.fvattn_hilbert_table.restype = _c_int
 _lib.fvattn_workspace_status.argtypes = [_c_void_p, _c_void_p]
 _lib.fvattn_workspace_status.restype = _c_int
+_lib.fvattn_wait_selftest.argtypes = [_c_void_p, _c_void_p, _c_size_t, _c_void_p]
+_lib.fvattn_wait_selftest.restype = _c_int
 _lib.fvattn_status_string.argtypes = [_c_int]
 _lib.fvattn_status_string.restype = ctypes.c_char_p
 
@@ -157,9 +160,50 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
-    s = stream if stream is not None else torch.cuda.current_stream()
+def _stream(stream, device=None):
+    """The given stream (which must belong to ``device``), else ``device``'s current stream."""
+    if stream is None:
+        s = torch.cuda.current_stream(device)
+    else:
+        s = stream
+        if device is not None and s.device != torch.device(device):
+            raise ValueError(f"stream is on {s.device}, tensors on {device}")
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def _expect(t, name, dev, shape=None, dtype=None, optional=False):
+    """Every buffer handed to the library: a contiguous CUDA tensor on ``dev`` with the
+    shape and dtype the C call assumes (the library sees only a pointer, so a wrong size
+    would make a kernel read or write past the end of the buffer)."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.device != dev:
+        raise ValueError(f"{name} is on {t.device}, expected {dev}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _expect_ws(ws, dev):
+    _expect(ws, "workspace", dev)
+
+
+def _call(dev, fn, *args):
+    """Runs a library call with ``dev`` current, so that device-side lookups (SM count,
+    static scratch) and launches happen on the tensors' device."""
+    with torch.cuda.device(dev):
+        return fn(*args)
+
+
+def _nb(N, block):
+    return -(-int(N) // int(block))
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -183,9 +227,14 @@ def fvattn_workspace_bytes(op: int, B: int, H: int, N: int, d: int, block: int) 
 def fvattn_permute(x, y, grid: Grid, inverse: bool = False, stream=None):
     """x [B,H,N,d] -> y [B,H,Npad,d] (tile order), or the inverse."""
     _need_cuda(x, y)
-    B, H, _, d = x.shape
-    _check(_lib.fvattn_permute(_ptr(x), _ptr(y), B, H, grid.N, d, _dtype_code(x), ctypes.byref(grid),
-                               1 if inverse else 0, _stream(stream)), "fvattn_permute")
+    dev = x.device
+    B, H, n_in, d = x.shape
+    npad = grid.nb * grid.block
+    if n_in != (npad if inverse else grid.N):
+        raise ValueError(f"x has {n_in} rows, expected {npad if inverse else grid.N}")
+    _expect(y, "y", dev, (B, H, grid.N if inverse else npad, d), x.dtype)
+    _check(_call(dev, _lib.fvattn_permute, _ptr(x), _ptr(y), B, H, grid.N, d, _dtype_code(x),
+                 ctypes.byref(grid), 1 if inverse else 0, _stream(stream, dev)), "fvattn_permute")
     return y
 
 
@@ -193,13 +242,35 @@ def fvattn_route(q, k, grid: Grid, p: float, k_min: int, kv_idx, kv_cnt, head_wo
                  qp_out=None, kp_out=None, stream=None):
     """Routing front end; fills kv_idx [B,H,nb,nb], kv_cnt [B,H,nb], head_work [B,H]."""
     _need_cuda(q, k, kv_idx, kv_cnt, head_work, workspace, qp_out, kp_out)
+    dev = q.device
     B, H, N, d = q.shape
-    _check(_lib.fvattn_route(_ptr(q), _ptr(k), B, H, N, d, _dtype_code(q), ctypes.byref(grid),
-                             float(p), int(k_min), _ptr(qp_out), _ptr(kp_out), _ptr(kv_idx),
-                             _ptr(kv_cnt), _ptr(head_work), _ptr(workspace),
-                             workspace.numel() * workspace.element_size(), _stream(stream)),
+    _check_route_buffers(q, k, grid, kv_idx, kv_cnt, head_work, qp_out, kp_out)
+    _expect_ws(workspace, dev)
+    _check(_call(dev, _lib.fvattn_route, _ptr(q), _ptr(k), B, H, N, d, _dtype_code(q), ctypes.byref(grid),
+                 float(p), int(k_min), _ptr(qp_out), _ptr(kp_out), _ptr(kv_idx),
+                 _ptr(kv_cnt), _ptr(head_work), _ptr(workspace),
+                 workspace.numel() * workspace.element_size(), _stream(stream, dev)),
            "fvattn_route")
     return kv_idx, kv_cnt, head_work
+
+
+def _check_lists(kv_idx, kv_cnt, head_work, dev, B, H, nb):
+    _expect(kv_idx, "kv_idx", dev, (B, H, nb, nb), torch.int32)
+    _expect(kv_cnt, "kv_cnt", dev, (B, H, nb), torch.int32)
+    _expect(head_work, "head_work", dev, (B, H), torch.int64, optional=head_work is None)
+
+
+def _check_route_buffers(q, k, grid, kv_idx, kv_cnt, head_work, qp_out, kp_out):
+    dev = q.device
+    B, H, N, d = q.shape
+    if N != grid.N:
+        raise ValueError(f"q has {N} tokens, the grid {grid.N}")
+    _dtype_code(q)
+    _expect(k, "k", dev, q.shape, q.dtype)
+    nb = grid.nb
+    _check_lists(kv_idx, kv_cnt, head_work, dev, B, H, nb)
+    for t, name in ((qp_out, "qp_out"), (kp_out, "kp_out")):
+        _expect(t, name, dev, (B, H, nb * grid.block, d), q.dtype, optional=True)
 
 
 def fvattn_route_noalloc(q, k, grid: Grid, p: float, k_min: int, kv_idx, kv_cnt, head_work,
@@ -208,12 +279,34 @@ def fvattn_route_noalloc(q, k, grid: Grid, p: float, k_min: int, kv_idx, kv_cnt,
     memory where they route; the library's static 96 MiB device scratch is used
     instead (calls that overlap on the GPU race on it)."""
     _need_cuda(q, k, kv_idx, kv_cnt, head_work, qp_out, kp_out)
+    dev = q.device
     B, H, N, d = q.shape
-    _check(_lib.fvattn_route_noalloc(_ptr(q), _ptr(k), B, H, N, d, _dtype_code(q), ctypes.byref(grid),
-                                     float(p), int(k_min), _ptr(qp_out), _ptr(kp_out), _ptr(kv_idx),
-                                     _ptr(kv_cnt), _ptr(head_work), _stream(stream)),
+    _check_route_buffers(q, k, grid, kv_idx, kv_cnt, head_work, qp_out, kp_out)
+    _check(_call(dev, _lib.fvattn_route_noalloc, _ptr(q), _ptr(k), B, H, N, d, _dtype_code(q),
+                 ctypes.byref(grid), float(p), int(k_min), _ptr(qp_out), _ptr(kp_out), _ptr(kv_idx),
+                 _ptr(kv_cnt), _ptr(head_work), _stream(stream, dev)),
            "fvattn_route_noalloc")
     return kv_idx, kv_cnt, head_work
+
+
+def _check_attn(qp, kp, v, out, N, block, workspace, lse, block_lse, v_dtype=None, vscale=None):
+    """Shapes of an attention call: qp, kp, out [B,H,Npad,d] of one dtype; v the same
+    shape (bf16/fp32 like qp, or E4M3 codes as uint8 with vscale [B,H,d] fp32);
+    lse [B,H,Npad] and block_lse [B,H,nb,Npad] fp32 when given."""
+    dev = qp.device
+    B, H, npad, d = qp.shape
+    nb = _nb(N, block)
+    if npad != nb * block:
+        raise ValueError(f"qp has {npad} rows, expected {nb * block} (N={N}, block={block})")
+    _dtype_code(qp)
+    _expect(kp, "kp", dev, qp.shape, qp.dtype)
+    _expect(v, "v", dev, qp.shape, v_dtype or qp.dtype)
+    _expect(out, "out", dev, qp.shape, qp.dtype)
+    _expect(vscale, "vscale", dev, (B, H, d), torch.float32, optional=vscale is None)
+    _expect(lse, "lse", dev, (B, H, npad), torch.float32, optional=True)
+    _expect(block_lse, "block_lse", dev, (B, H, nb, npad), torch.float32, optional=True)
+    _expect_ws(workspace, dev)
+    return dev, B, H, d, nb
 
 
 def fvattn_sparse_fwd(qp, kp, vp, out, kv_idx, kv_cnt, N: int, block: int, workspace,
@@ -221,12 +314,13 @@ def fvattn_sparse_fwd(qp, kp, vp, out, kv_idx, kv_cnt, N: int, block: int, works
     """Block-sparse attention over permuted [B,H,Npad,d] tensors; optional lse
     [B,H,Npad] and block_lse [B,H,nb,Npad] (fp32) outputs."""
     _need_cuda(qp, kp, vp, out, kv_idx, kv_cnt, workspace, lse, block_lse)
-    B, H, _, d = qp.shape
+    dev, B, H, d, nb = _check_attn(qp, kp, vp, out, N, block, workspace, lse, block_lse)
+    _check_lists(kv_idx, kv_cnt, None, dev, B, H, nb)
     sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    _check(_lib.fvattn_sparse_fwd(_ptr(qp), _ptr(kp), _ptr(vp), _ptr(out), _ptr(lse), _ptr(block_lse),
-                                  _ptr(kv_idx), _ptr(kv_cnt), B, H, N, d, _dtype_code(qp), block, sc,
-                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                  _stream(stream)), "fvattn_sparse_fwd")
+    _check(_call(dev, _lib.fvattn_sparse_fwd, _ptr(qp), _ptr(kp), _ptr(vp), _ptr(out), _ptr(lse),
+                 _ptr(block_lse), _ptr(kv_idx), _ptr(kv_cnt), B, H, N, d, _dtype_code(qp), block, sc,
+                 _ptr(workspace), workspace.numel() * workspace.element_size(),
+                 _stream(stream, dev)), "fvattn_sparse_fwd")
     return out
 
 
@@ -234,12 +328,11 @@ def fvattn_dense_fwd(qp, kp, vp, out, N: int, block: int, workspace, scale=None,
                      block_lse=None, stream=None):
     """Dense attention over permuted [B,H,Npad,d] tensors (every key block)."""
     _need_cuda(qp, kp, vp, out, workspace, lse, block_lse)
-    B, H, _, d = qp.shape
+    dev, B, H, d, nb = _check_attn(qp, kp, vp, out, N, block, workspace, lse, block_lse)
     sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    _check(_lib.fvattn_dense_fwd(_ptr(qp), _ptr(kp), _ptr(vp), _ptr(out), _ptr(lse), _ptr(block_lse),
-                                 B, H, N, d,
-                                 _dtype_code(qp), block, sc, _ptr(workspace),
-                                 workspace.numel() * workspace.element_size(), _stream(stream)),
+    _check(_call(dev, _lib.fvattn_dense_fwd, _ptr(qp), _ptr(kp), _ptr(vp), _ptr(out), _ptr(lse),
+                 _ptr(block_lse), B, H, N, d, _dtype_code(qp), block, sc, _ptr(workspace),
+                 workspace.numel() * workspace.element_size(), _stream(stream, dev)),
            "fvattn_dense_fwd")
     return out
 
@@ -248,11 +341,17 @@ def fvattn_quantize_v(vp, vq, vscale, N: int, block: int, workspace, stream=None
     """Per-channel E4M3 quantization: vp [B,H,Npad,128] bf16 -> vq [B,H,Npad,128]
     uint8 codes and vscale [B,H,128] fp32."""
     _need_cuda(vp, vq, vscale, workspace)
-    B, H, _, d = vp.shape
+    dev = vp.device
+    B, H, npad, d = vp.shape
     if vp.dtype != torch.bfloat16 or vq.dtype != torch.uint8 or vscale.dtype != torch.float32:
         raise TypeError("vp bf16, vq uint8, vscale float32")
-    _check(_lib.fvattn_quantize_v(_ptr(vp), B, H, N, d, block, _ptr(vq), _ptr(vscale), _ptr(workspace),
-                                  workspace.numel() * workspace.element_size(), _stream(stream)),
+    if npad != _nb(N, block) * block:
+        raise ValueError(f"vp has {npad} rows, expected {_nb(N, block) * block}")
+    _expect(vq, "vq", dev, vp.shape, torch.uint8)
+    _expect(vscale, "vscale", dev, (B, H, d), torch.float32)
+    _expect_ws(workspace, dev)
+    _check(_call(dev, _lib.fvattn_quantize_v, _ptr(vp), B, H, N, d, block, _ptr(vq), _ptr(vscale),
+                 _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream, dev)),
            "fvattn_quantize_v")
     return vq, vscale
 
@@ -261,12 +360,14 @@ def fvattn_sparse_fwd_fp8v(qp, kp, vq, vscale, out, kv_idx, kv_cnt, N: int, bloc
                            scale=None, lse=None, block_lse=None, stream=None):
     """fvattn_sparse_fwd with the E4M3 V of fvattn_quantize_v (8-bit P.V product)."""
     _need_cuda(qp, kp, vq, vscale, out, kv_idx, kv_cnt, workspace, lse, block_lse)
-    B, H, _, d = qp.shape
+    dev, B, H, d, nb = _check_attn(qp, kp, vq, out, N, block, workspace, lse, block_lse,
+                                   v_dtype=torch.uint8, vscale=vscale)
+    _check_lists(kv_idx, kv_cnt, None, dev, B, H, nb)
     sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    _check(_lib.fvattn_sparse_fwd_fp8v(_ptr(qp), _ptr(kp), _ptr(vq), _ptr(vscale), _ptr(out), _ptr(lse),
-                                       _ptr(block_lse), _ptr(kv_idx), _ptr(kv_cnt), B, H, N, d, block, sc,
-                                       _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                       _stream(stream)), "fvattn_sparse_fwd_fp8v")
+    _check(_call(dev, _lib.fvattn_sparse_fwd_fp8v, _ptr(qp), _ptr(kp), _ptr(vq), _ptr(vscale), _ptr(out),
+                 _ptr(lse), _ptr(block_lse), _ptr(kv_idx), _ptr(kv_cnt), B, H, N, d, block, sc,
+                 _ptr(workspace), workspace.numel() * workspace.element_size(),
+                 _stream(stream, dev)), "fvattn_sparse_fwd_fp8v")
     return out
 
 
@@ -274,11 +375,12 @@ def fvattn_dense_fwd_fp8v(qp, kp, vq, vscale, out, N: int, block: int, workspace
                           block_lse=None, stream=None):
     """fvattn_dense_fwd with the E4M3 V of fvattn_quantize_v (8-bit P.V product)."""
     _need_cuda(qp, kp, vq, vscale, out, workspace, lse, block_lse)
-    B, H, _, d = qp.shape
+    dev, B, H, d, nb = _check_attn(qp, kp, vq, out, N, block, workspace, lse, block_lse,
+                                   v_dtype=torch.uint8, vscale=vscale)
     sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    _check(_lib.fvattn_dense_fwd_fp8v(_ptr(qp), _ptr(kp), _ptr(vq), _ptr(vscale), _ptr(out), _ptr(lse),
-                                      _ptr(block_lse), B, H, N, d, block, sc, _ptr(workspace),
-                                      workspace.numel() * workspace.element_size(), _stream(stream)),
+    _check(_call(dev, _lib.fvattn_dense_fwd_fp8v, _ptr(qp), _ptr(kp), _ptr(vq), _ptr(vscale), _ptr(out),
+                 _ptr(lse), _ptr(block_lse), B, H, N, d, block, sc, _ptr(workspace),
+                 workspace.numel() * workspace.element_size(), _stream(stream, dev)),
            "fvattn_dense_fwd_fp8v")
     return out
 
@@ -288,10 +390,21 @@ def fvattn_block_importance(block_lse, lse, importance, N: int, block: int, work
     """Exact block importance [B,H,nb,nb] from an attention call's block_lse and lse
     (kv_idx/kv_cnt: the call's lists; None for a dense call)."""
     _need_cuda(block_lse, lse, importance, workspace, kv_idx, kv_cnt)
+    dev = lse.device
     B, H = lse.shape[:2]
-    _check(_lib.fvattn_block_importance(_ptr(block_lse), _ptr(lse), _ptr(kv_idx), _ptr(kv_cnt), B, H,
-                                        N, block, _ptr(importance), _ptr(workspace),
-                                        workspace.numel() * workspace.element_size(), _stream(stream)),
+    nb = _nb(N, block)
+    npad = nb * block
+    _expect(lse, "lse", dev, (B, H, npad), torch.float32)
+    _expect(block_lse, "block_lse", dev, (B, H, nb, npad), torch.float32)
+    _expect(importance, "importance", dev, (B, H, nb, nb), torch.float32)
+    if (kv_idx is None) != (kv_cnt is None):
+        raise ValueError("kv_idx and kv_cnt go together")
+    if kv_idx is not None:
+        _check_lists(kv_idx, kv_cnt, None, dev, B, H, nb)
+    _expect_ws(workspace, dev)
+    _check(_call(dev, _lib.fvattn_block_importance, _ptr(block_lse), _ptr(lse), _ptr(kv_idx), _ptr(kv_cnt),
+                 B, H, N, block, _ptr(importance), _ptr(workspace),
+                 workspace.numel() * workspace.element_size(), _stream(stream, dev)),
            "fvattn_block_importance")
     return importance
 
@@ -300,10 +413,16 @@ def fvattn_attention_recall(importance, kv_idx, kv_cnt, recall, N: int, block: i
                             stream=None):
     """Per query block, the dense importance captured by the lists: recall [B,H,nb]."""
     _need_cuda(importance, kv_idx, kv_cnt, recall, workspace)
+    dev = kv_cnt.device
     B, H = kv_cnt.shape[:2]
-    _check(_lib.fvattn_attention_recall(_ptr(importance), _ptr(kv_idx), _ptr(kv_cnt), B, H, N, block,
-                                        _ptr(recall), _ptr(workspace),
-                                        workspace.numel() * workspace.element_size(), _stream(stream)),
+    nb = _nb(N, block)
+    _check_lists(kv_idx, kv_cnt, None, dev, B, H, nb)
+    _expect(importance, "importance", dev, (B, H, nb, nb), torch.float32)
+    _expect(recall, "recall", dev, (B, H, nb), torch.float32)
+    _expect_ws(workspace, dev)
+    _check(_call(dev, _lib.fvattn_attention_recall, _ptr(importance), _ptr(kv_idx), _ptr(kv_cnt), B, H, N,
+                 block, _ptr(recall), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                 _stream(stream, dev)),
            "fvattn_attention_recall")
     return recall
 
@@ -312,10 +431,15 @@ def fvattn_select_topp(importance, N: int, block: int, p: float, k_min: int, kv_
                        workspace, stream=None):
     """Top-p + Top-k floor on importance rows [B,H,nb,nb] (the GSRS search over a candidate set)."""
     _need_cuda(importance, kv_idx, kv_cnt, head_work, workspace)
+    dev = kv_cnt.device
     B, H = kv_cnt.shape[:2]
-    _check(_lib.fvattn_select_topp(_ptr(importance), B, H, N, block, float(p), int(k_min), _ptr(kv_idx),
-                                   _ptr(kv_cnt), _ptr(head_work), _ptr(workspace),
-                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+    nb = _nb(N, block)
+    _check_lists(kv_idx, kv_cnt, head_work, dev, B, H, nb)
+    _expect(importance, "importance", dev, (B, H, nb, nb), torch.float32)
+    _expect_ws(workspace, dev)
+    _check(_call(dev, _lib.fvattn_select_topp, _ptr(importance), B, H, N, block, float(p), int(k_min),
+                 _ptr(kv_idx), _ptr(kv_cnt), _ptr(head_work), _ptr(workspace),
+                 workspace.numel() * workspace.element_size(), _stream(stream, dev)),
            "fvattn_select_topp")
     return kv_idx, kv_cnt, head_work
 
@@ -324,10 +448,13 @@ def fvattn_lvsa_lists(grid: Grid, window: int, period: int, step: int, kv_idx, k
                       workspace, stream=None):
     """LVSA window + rotating global-frame lists for every (b, h) of kv_cnt's [B,H,nb] shape."""
     _need_cuda(kv_idx, kv_cnt, head_work, workspace)
+    dev = kv_cnt.device
     B, H = kv_cnt.shape[:2]
-    _check(_lib.fvattn_lvsa_lists(B, H, ctypes.byref(grid), int(window), int(period), int(step),
-                                  _ptr(kv_idx), _ptr(kv_cnt), _ptr(head_work), _ptr(workspace),
-                                  workspace.numel() * workspace.element_size(), _stream(stream)),
+    _check_lists(kv_idx, kv_cnt, head_work, dev, B, H, grid.nb)
+    _expect_ws(workspace, dev)
+    _check(_call(dev, _lib.fvattn_lvsa_lists, B, H, ctypes.byref(grid), int(window), int(period), int(step),
+                 _ptr(kv_idx), _ptr(kv_cnt), _ptr(head_work), _ptr(workspace),
+                 workspace.numel() * workspace.element_size(), _stream(stream, dev)),
            "fvattn_lvsa_lists")
     return kv_idx, kv_cnt, head_work
 
@@ -338,17 +465,32 @@ def fvattn_hilbert_table(grid_thw, block: int = 128, device="cuda", stream=None)
     g = Grid(T, Hh, W, 1, 1, 1, block, FVATTN_ORDER_TILES, None)
     N = T * Hh * W
     table = torch.empty(N, dtype=torch.int32, device=device)
-    ws = alloc_workspace(fvattn_workspace_bytes(FVATTN_OP_HILBERT, 1, 1, N, 64, block), device)
-    _check(_lib.fvattn_hilbert_table(ctypes.byref(g), _ptr(table), _ptr(ws),
-                                     ws.numel() * ws.element_size(), _stream(stream)),
+    dev = table.device
+    ws = alloc_workspace(fvattn_workspace_bytes(FVATTN_OP_HILBERT, 1, 1, N, 64, block), dev)
+    _check(_call(dev, _lib.fvattn_hilbert_table, ctypes.byref(g), _ptr(table), _ptr(ws),
+                 ws.numel() * ws.element_size(), _stream(stream, dev)),
            "fvattn_hilbert_table")
-    torch.cuda.current_stream(device).synchronize() if stream is None else stream.synchronize()
+    torch.cuda.current_stream(dev).synchronize() if stream is None else stream.synchronize()
     return table
 
 
 def fvattn_workspace_status(workspace, stream=None) -> int:
     """Synchronize the stream and return the status word the kernels recorded."""
-    return int(_lib.fvattn_workspace_status(_ptr(workspace), _stream(stream)))
+    _need_cuda(workspace)
+    dev = workspace.device
+    return int(_call(dev, _lib.fvattn_workspace_status, _ptr(workspace), _stream(stream, dev)))
+
+
+def fvattn_wait_selftest(results, workspace, stream=None):
+    """Runs the bounded-wait self-test (no fault: waits on barriers nothing arrives at);
+    results [8] int64 on the device. The status word then reads FVATTN_ERR_TIMEOUT."""
+    _need_cuda(results, workspace)
+    dev = results.device
+    _expect(results, "results", dev, (8,), torch.int64)
+    _expect_ws(workspace, dev)
+    _check(_call(dev, _lib.fvattn_wait_selftest, _ptr(results), _ptr(workspace),
+                 workspace.numel() * workspace.element_size(), _stream(stream, dev)), "fvattn_wait_selftest")
+    return results
 
 
 def alloc_workspace(nbytes: int, device) -> torch.Tensor:

@@ -45,6 +45,7 @@ cudaError_t launch_hilbert_table(int T, int Hh, int W, int* table, unsigned long
 cudaError_t launch_quantize_v(const void* v, int BH, int N, int npad, uint8_t* vq, float* vscale,
                               unsigned int* amax_bits, cudaStream_t st);
 size_t vquant_ws_bytes(int BH);
+cudaError_t launch_wait_selftest(long long* out, int* status, cudaStream_t st);
 int hilbert_bits(int extent);
 int next_pow2(int n);
 }  // namespace fvattn
@@ -501,6 +502,18 @@ fvattn_status fvattn_hilbert_table(const fvattn_grid* grid, int32_t* table, void
   if (cudaMemsetAsync(base, 0, kWsHeaderBytes, st) != cudaSuccess) return FVATTN_ERR_CUDA;
   return from_cuda(fvattn::launch_hilbert_table(
       grid->T, grid->Hh, grid->W, table, reinterpret_cast<unsigned long long*>(base + kWsHeaderBytes), st));
+}
+
+fvattn_status fvattn_wait_selftest(int64_t* results, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  if (!results || !aligned(results, 8)) return FVATTN_ERR_INVALID_ARG;
+  const fvattn_status wst = check_ws(workspace, workspace_bytes, kWsHeaderBytes);
+  if (wst != FVATTN_OK) return wst;
+  auto st = static_cast<cudaStream_t>(stream);
+  auto hdr = static_cast<fvattn::WsHeader*>(workspace);
+  if (cudaMemsetAsync(workspace, 0, kWsHeaderBytes, st) != cudaSuccess) return FVATTN_ERR_CUDA;
+  if (cudaMemsetAsync(results, 0, 8 * sizeof(int64_t), st) != cudaSuccess) return FVATTN_ERR_CUDA;
+  return from_cuda(fvattn::launch_wait_selftest(reinterpret_cast<long long*>(results), &hdr->status, st));
 }
 
 fvattn_status fvattn_workspace_status(const void* workspace, void* stream) {

@@ -77,12 +77,6 @@ constexpr int kThreads = 384;
 constexpr int kRegsSoftmax = 184;
 constexpr int kRegsControl = 128;
 constexpr float kLn2 = 0.6931471805599453f;
-// One in kPolyEvery exponential pairs runs on the FMA pipe (exp2_poly3), the
-// rest on MUFU; 0 keeps every exponential on MUFU.
-#ifndef FVATTN_POLY_EVERY
-#define FVATTN_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = FVATTN_POLY_EVERY;
 
 // A step covers 128 keys: one 128-token block, or two consecutive union entries
 // of 64-token blocks whose K (V) tiles are loaded into the two 64-row halves of
@@ -223,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm.abort_flag = 0;
     fence_mbarrier_init();
   }
-  if (warp == 9) {
+  if (warp == 9) {   // warp-uniform: the whole warp allocates
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
@@ -238,11 +232,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
 
   // All 384 threads meet here once at the end; then the allocating warp frees TMEM.
+  //
+  // Warp-collective tensor-memory instructions (tcgen05.alloc/dealloc/ld/st and
+  // wait::ld/st, all .sync.aligned) must be executed by every lane of the warp
+  // together. Each call site below states why its control flow is warp-uniform.
+  // The %globaltimer bound on the mbarrier waits cannot rescue a warp whose lanes
+  // diverged around such an instruction: the lanes that reached it wait there for
+  // the others with no limit. (An earlier version rescaled O under a per-row
+  // branch around tcgen05.ld/st; a first test run with large logits hung in it
+  // until the run was killed. The rescale now branches on a warp vote.)
   auto teardown = [&]() {
     __syncwarp();
     tc_fence_before();
     asm volatile("barrier.sync 1, %0;" ::"n"(kThreads) : "memory");
-    if (warp == 9) {
+    if (warp == 9) {   // warp-uniform: every lane of warp 9 passed the barrier above
       __syncwarp();
       tc_fence_after();
       tmem_dealloc(tmem, 512);
@@ -456,6 +459,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mem[h] = (e[h] >> (16 + qb)) & 1u;     // warp-uniform: a warp's rows share qb
           any_mem |= mem[h];
         }
+        // any_mem is warp-uniform: it depends only on the step's union entries
+        // (the same for every lane) and on qb, which all 32 rows of a warp share
+        // (32 divides BN). The S loads and P stores below therefore run on full warps.
         if (any_mem) {
           uint32_t s[NC][32];
 #pragma unroll
@@ -537,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // any row of the warp needs a larger max, the whole warp rescales,
             // rows that do not need it with factor 1.
             const bool need = m_new > m_run + T::kThreshold;
-            if (__any_sync(0xffffffffu, need)) {
+            if (__any_sync(0xffffffffu, need)) {   // vote: the O load/store below is warp-uniform
               const float f = need ? ex2_approx(m_run - m_new) : 1.f;
               l_run *= f;
 #pragma unroll 1
@@ -571,15 +577,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 16; ++i) {
               const float2 xv = __ffma2_rn(
                   make_float2(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])), sl2x2, negc);
-              float p0, p1;
-              if (kPolyEvery > 0 && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
-                const float2 pv = exp2_poly3x2(xv);
-                p0 = pv.x;
-                p1 = pv.y;
-              } else {
-                p0 = ex2_approx(xv.x);
-                p1 = ex2_approx(xv.y);
-              }
+              const float p0 = ex2_approx(xv.x);
+              const float p1 = ex2_approx(xv.y);
               if constexpr (F8) {
                 // four keys per 32-bit word, lowest key in the low byte
                 const uint32_t q8 = pack_e4m3x2(p0, p1);
@@ -597,7 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               lc[c] = __fadd2_rn(ls[0], ls[1]);
               tmem_st16(tS + c * 16, pk);
             }
-            if (c == NC / 2 - 1 || c == NC - 1) {
+            if (c == NC / 2 - 1 || c == NC - 1) {   // c is a compile-time loop index: uniform
               tmem_wait_st();
               tc_fence_before();
               __syncwarp();
@@ -617,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               P.blse[(static_cast<size_t>(x.bh) * P.nb + (e[h] & 0xFFFFu)) * P.npad + qrow] =
                   (m_eff + __log2f(l_blk)) * kLn2;
           }
-        } else {
+        } else {   // the same warp-uniform condition, negated: P = 0 for the whole step
           uint32_t z[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) z[i] = 0u;
@@ -638,7 +637,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       // Rows past the head's last block (the second half of a 64-token-block
       // tile at the end of a head) are not stored; the TMEM loads stay
-      // warp-collective.
+      // warp-collective (the loop runs for every lane; `store` only guards the
+      // global stores). Every exit above is a warp-wide vote (__all_sync) or a
+      // value read from shared memory by all lanes (the unit, its slots).
       const bool store = qrow < P.npad;
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
       const float* vs = F8 ? P.vscale + static_cast<size_t>(x.bh) * HD : nullptr;

@@ -22,10 +22,15 @@
 //     several host threads) race on the array: keep them ordered.
 //   - The array's device address is looked up with cudaGetSymbolAddress on the
 //     first call on each device (with that device current) and cached; make
-//     that first call before capturing a stream into a graph.
+//     that first call before capturing a stream into a graph. The cache is
+//     keyed on the CUDA context that was current at the lookup: a call under
+//     another context (cudaDeviceReset made a new primary context, or the
+//     caller made a context of its own current) looks the address up again, so
+//     such a first call under a new context should also come before any capture.
 //   - Nothing here allocates: no cudaMalloc, no cudaFree, no allocating
 //     library routine.
-#include <atomic>
+#include <cuda.h>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -36,19 +41,48 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char fvattn_route_scratch[kScratchBytes];
 
-std::atomic<void*> g_scratch[kMaxDevices];
+// The driver's cuCtxGetCurrent, looked up once through the runtime (the library
+// does not link libcuda directly).
+using CtxGetCurrent = CUresult (*)(CUcontext*);
+CtxGetCurrent ctx_get_current() {
+  static const CtxGetCurrent fn = []() -> CtxGetCurrent {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<CtxGetCurrent>(p);
+    return nullptr;
+  }();
+  return fn;
+}
 
-// Device address of the scratch array on the current device (nullptr on error).
+CUcontext current_context() {
+  CUcontext c = nullptr;
+  const CtxGetCurrent f = ctx_get_current();
+  if (!f || f(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+struct CacheEntry {
+  CUcontext ctx;
+  void* ptr;
+};
+std::mutex g_mu;
+CacheEntry g_cache[kMaxDevices];
+
+// Device address of the scratch array in the current device's current context
+// (nullptr on error). Calls from several host threads are serialised by g_mu.
 void* scratch_on_current_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return nullptr;
-  if (dev < kMaxDevices) {
-    void* cached = g_scratch[dev].load(std::memory_order_acquire);
-    if (cached) return cached;
-  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  CUcontext ctx = current_context();
+  if (dev < kMaxDevices && ctx && g_cache[dev].ctx == ctx && g_cache[dev].ptr) return g_cache[dev].ptr;
   void* ptr = nullptr;
   if (cudaGetSymbolAddress(&ptr, fvattn_route_scratch) != cudaSuccess || !ptr) return nullptr;
-  if (dev < kMaxDevices) g_scratch[dev].store(ptr, std::memory_order_release);
+  ctx = current_context();    // the lookup makes the device's primary context current if none was
+  if (dev < kMaxDevices && ctx) g_cache[dev] = CacheEntry{ctx, ptr};
   return ptr;
 }
 

@@ -258,28 +258,6 @@ __device__ __forceinline__ void regs_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-// 2^x for two values on the FMA pipe, to take part of the softmax's
-// exponentials off the MUFU unit. Cody-Waite style range reduction x = n + f
-// with n = round(x) (obtained by adding 1.5 * 2^23, which leaves n in the low
-// mantissa bits) and f in [-1/2, 1/2]; 2^f by a cubic whose coefficients were
-// fitted for minimal relative error by a Remez exchange (max relative error
-// 7.5e-5, far below the 2^-9 of the bf16 that P is rounded to); 2^n is added
-// to the exponent field. Inputs are clamped to >= -126, so -inf gives 2^-126,
-// which is zero for every purpose here (P <= 2^8, row sums >= 1).
-__device__ __forceinline__ float2 exp2_poly3x2(float2 x) {
-  constexpr float kC0 = 0.99992806f, kC1 = 0.69326097f, kC2 = 0.24261113f, kC3 = 0.05517167f;
-  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
-  const float2 xc = make_float2(fmaxf(x.x, -126.0f), fmaxf(x.y, -126.0f));
-  const float2 t = __fadd2_rn(xc, make_float2(kMagic, kMagic));
-  const float2 n = __fadd2_rn(t, make_float2(-kMagic, -kMagic));
-  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), xc);
-  float2 p = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
-  p = __ffma2_rn(p, f, make_float2(kC1, kC1));
-  p = __ffma2_rn(p, f, make_float2(kC0, kC0));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));

@@ -169,8 +169,12 @@ FVATTN_API fvattn_status fvattn_route(const void* q, const void* k, int B, int H
  * library keeps until exit. Sizes whose route workspace exceeds 96 MiB return
  * FVATTN_ERR_WORKSPACE and launch nothing. All calls on a device share the
  * array, so calls that overlap on the GPU race; the first call on each device
- * looks up the array's address (do it before any stream capture). Nothing is
- * allocated. Kernel-side status words are not reported by this variant. */
+ * looks up the array's address (do it before any stream capture). The address
+ * is cached per device and per CUDA context: a call under a context other than
+ * the one of that lookup (after cudaDeviceReset, or with a caller-made context
+ * current) looks it up again, and that call too belongs before any capture.
+ * Nothing is allocated. Kernel-side status words are not reported by this
+ * variant. */
 FVATTN_API fvattn_status fvattn_route_noalloc(const void* q, const void* k, int B, int H, int N,
                                               int d, fvattn_dtype dtype, const fvattn_grid* grid,
                                               float p, int k_min, void* qp_out, void* kp_out,
@@ -205,8 +209,11 @@ FVATTN_API fvattn_status fvattn_sparse_fwd(const void* qp, const void* kp, const
                                 void* workspace, size_t workspace_bytes,
                                 void* stream);
 
-/* Dense attention forward: fvattn_sparse_fwd with every key block selected
- * (block_lse, when given, is written for every (row, key block) pair).
+/* Dense attention forward [FVAttn §4.1: dense FlashAttention is the 1.00x
+ * baseline of every latency table]: fvattn_sparse_fwd with every key block
+ * selected, on the same kernels (block_lse, when given, is written for every
+ * (row, key block) pair). Same arguments, layouts, ownership and errors as
+ * fvattn_sparse_fwd without kv_idx/kv_cnt.
  * Workspace: fvattn_workspace_bytes(FVATTN_OP_DENSE_FWD, ...). */
 FVATTN_API fvattn_status fvattn_dense_fwd(const void* qp, const void* kp, const void* vp,
                                void* op, float* lse, float* block_lse, int B, int H, int N,
@@ -341,6 +348,26 @@ FVATTN_API fvattn_status fvattn_lvsa_lists(int B, int H, const fvattn_grid* grid
 /* Synchronizes `stream` and returns the status word that the kernels of the
  * last call using `workspace` recorded (FVATTN_OK if none). */
 FVATTN_API fvattn_status fvattn_workspace_status(const void* workspace, void* stream);
+
+/* Self-test of the bounded device waits (failure detection; the pages have no
+ * counterpart: their runtime balances stragglers but detects no faults).
+ * Every wait of the library's kernels on an mbarrier gives up after a fixed
+ * limit of the GPU's global timer (2 s), raises an abort flag that releases
+ * every other waiter of the block, and records FVATTN_ERR_TIMEOUT in the
+ * workspace status word, so a lost arrival ends the kernel instead of hanging
+ * the GPU. This call runs those waits on barriers that nothing arrives at: one
+ * block of 64 threads, no other memory touched. After the stream reaches it
+ * (about two limits, 4 s), fvattn_workspace_status reads FVATTN_ERR_TIMEOUT and
+ * the device context is still usable.
+ *   results  [8] int64, device, written: [0] 1 if the first wait succeeded
+ *            (expected 0), [1] its duration in ns (about the limit), [2] and [3]
+ *            the same for a wait in another warp released by the abort flag,
+ *            [4] and [5] for the final-drain form of the wait (no abort flag),
+ *            [6] the limit in ns, [7] the abort flag (expected 1).
+ * Workspace: 256 bytes, 256-byte aligned (fvattn_workspace_bytes of
+ * FVATTN_OP_DENSE_FWD gives that size). Returns FVATTN_OK once launched. */
+FVATTN_API fvattn_status fvattn_wait_selftest(int64_t* results, void* workspace, size_t workspace_bytes,
+                                              void* stream);
 
 /* Static string for a status code (never NULL). */
 FVATTN_API const char* fvattn_status_string(fvattn_status status);

@@ -54,3 +54,9 @@ from .hilbert_oracle import (  # noqa: F401
     hilbert_index,
     hilbert_order,
 )
+from .mask_parity import (  # noqa: F401
+    BORDER_REL,
+    BORDER_CUM,
+    compare_masks,
+    borderline_ceiling,
+)

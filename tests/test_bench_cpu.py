@@ -59,3 +59,55 @@ def test_reference_arm_line(capsys):
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["value"] > 0
+
+
+def test_reference_arm_config_matches_the_gpu_arm(capsys):
+    rc = bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "3"])
+    assert rc == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["config"] == bench.bench_config(S.WORKLOADS["tiny"], 1)
+
+
+def test_hbm_bytes_of_the_720p_call():
+    w = S.WORKLOADS["wan14b-720p"]
+    nb = w.nb
+    hb = bench.hbm_bytes(w, nb, cnt_sum=1000)
+    R = 40 * 75600 * 128 * 2
+    P = 40 * nb * 128 * 128 * 2
+    assert hb["permute_v"] == R + P and hb["inverse"] == 2 * R
+    assert hb["route"] == 2 * R + 2 * P + 2 * 40 * nb * 128 * 4 + 4 * 1000 + 4 * 40 * nb
+    total = sum(hb.values()) / 1e9
+    assert 6.1 < total < 6.3
+
+
+def test_oracle_check_on_the_oracles_own_result():
+    """Lists and outputs taken from the oracle itself: no mismatch, zero error."""
+    import math
+
+    import numpy as np
+
+    import oracle as O
+    w = S.WORKLOADS["tiny"]
+    q, k, v = (x.numpy() for x in S.make_qkv(w, device="cpu"))
+    orc = O.route(q, k, w.grid6, w.block, w.p, w.k_min)
+    nb = w.nb
+    idx = np.zeros((w.B, w.H, nb, nb), dtype=np.int32)
+    for r in np.ndindex(*orc["cnt"].shape):
+        c = int(orc["cnt"][r])
+        idx[r][:c] = np.sort(orc["order"][r][:c])
+    cnt = orc["cnt"].astype(np.int32)
+    mask = O.selection_mask(orc["order"], orc["cnt"])
+    perm = orc["perm"]
+    op = O.masked_attention(*(O.permute(x, perm, w.block) for x in (q, k, v)), mask, w.N, w.block,
+                            1.0 / math.sqrt(w.d))
+    mp, err, route_s, attn_s, flops, blocks = bench.oracle_check(
+        w, q, k, v, idx, cnt, op, range(w.H), per_head=2, rng=np.random.default_rng(0))
+    assert mp["mismatched"] == 0 and mp["hard"] == 0 and mp["heads"] == w.H
+    assert mp["rows"] == w.H * nb and mp["selected_pairs"] == int(cnt.sum())
+    assert err["max_abs"] < 1e-12 and err["within_tolerance"] and blocks >= w.H
+    assert flops > 0 and route_s >= 0 and attn_s >= 0
+    # a planted wrong output row is seen
+    op[0, 0, 0, 0] += 1.0
+    rng = np.random.default_rng(0)
+    _, err2, *_ = bench.oracle_check(w, q, k, v, idx, cnt, op, [0], per_head=nb, rng=rng)
+    assert err2["max_abs"] >= 0.999 and not err2["within_tolerance"]

@@ -11,8 +11,8 @@ import torch
 
 import oracle as O
 import synthetic as S
-from parity import (BF16_MAX_ABS, BF16_MEAN_ABS, FP32_MAX_ABS, attention_errors, check_lists_valid,
-                    compare_masks, mask_from_lists)
+from parity import (BF16_MAX_ABS, BF16_MEAN_ABS, FP32_MAX_ABS, assert_mask_parity, attention_errors,
+                    check_lists_valid, compare_masks, mask_from_lists)
 
 pytestmark = pytest.mark.gpu
 
@@ -46,8 +46,7 @@ def test_degenerate_grids(w):
     orc = O.route(qn, kn, w.grid6, w.block, w.p, w.k_min)
     idx, cnt = path.kv_idx.cpu().numpy(), path.kv_cnt.cpu().numpy()
     check_lists_valid(idx, cnt, path.nb, w.k_min)
-    n_mis, _, hard = compare_masks(mask_from_lists(idx, cnt, path.nb), orc, w.p)
-    assert not hard, hard[:3]
+    assert_mask_parity(compare_masks(mask_from_lists(idx, cnt, path.nb), orc, w.p), w.name)
     mask = mask_from_lists(idx, cnt, path.nb)
     ref = O.masked_attention(*(O.permute(x, orc["perm"], w.block) for x in (qn, kn, vn)), mask, w.N,
                              w.block, 1.0 / math.sqrt(w.d))
@@ -72,8 +71,8 @@ def test_largest_supported_block_count():
     idx, cnt = path.kv_idx.cpu().numpy(), path.kv_cnt.cpu().numpy()
     check_lists_valid(idx, cnt, path.nb, w.k_min)
     mask = mask_from_lists(idx, cnt, path.nb)
-    n_mis, n_border, hard = compare_masks(mask, orc, w.p)
-    assert not hard, hard[:3]
+    mres = compare_masks(mask, orc, w.p)
+    assert_mask_parity(mres, w.name)
     perm = orc["perm"]
     qp, kp, vp = (O.permute(x[0, 0], perm, w.block) for x in (qn, kn, vn))
     outp = O.permute(out[0, 0], perm, w.block)
@@ -83,4 +82,39 @@ def test_largest_supported_block_count():
         got = outp[i * w.block:i * w.block + ref.shape[0]]
         mx, mean = attention_errors(got, ref)
         assert mx <= BF16_MAX_ABS and mean <= BF16_MEAN_ABS, (i, mx, mean)
-    print(f"max-blocks: nb={path.nb} density {mask.mean():.3f} mismatched={n_mis} borderline={n_border}")
+    print(f"max-blocks: nb={path.nb} density {mask.mean():.3f} mismatched={mres['mismatched']} "
+          f"borderline={mres['borderline']}")
+
+
+def test_binding_rejects_mismatched_buffers_before_any_launch():
+    """The binding checks every buffer's shape, dtype and device against the call (the
+    library itself sees only pointers)."""
+    w = S.Workload("bind", 1, 2, 128, "bf16", (2, 8, 15), (1, 8, 16), 128, 0.9, 1, seed=67)   # N=240, ragged
+    dev = torch.device("cuda")
+    q, k, v = S.make_qkv(w, device=dev)
+    grid = F.Grid.make(w.grid, w.tile, w.block)
+    nb, npad = grid.nb, grid.nb * w.block
+    idx = torch.empty((1, 2, nb, nb), dtype=torch.int32, device=dev)
+    cnt = torch.empty((1, 2, nb), dtype=torch.int32, device=dev)
+    hw = torch.empty((1, 2), dtype=torch.int64, device=dev)
+    ws = F.alloc_workspace(F.fvattn_workspace_bytes(F.FVATTN_OP_ROUTE, 1, 2, w.N, w.d, w.block), dev)
+    with pytest.raises(ValueError):      # list buffer one row short
+        F.fvattn_route(q, k, grid, 0.9, 1, idx[:, :, :, :-1].contiguous(), cnt, hw, ws)
+    with pytest.raises(TypeError):       # k in another dtype than q
+        F.fvattn_route(q, k.float(), grid, 0.9, 1, idx, cnt, hw, ws)
+    with pytest.raises(TypeError):       # counts in int64
+        F.fvattn_route(q, k, grid, 0.9, 1, idx, cnt.long(), hw, ws)
+    with pytest.raises(ValueError):      # permuted output without the pad rows
+        F.fvattn_route(q, k, grid, 0.9, 1, idx, cnt, hw, ws, qp_out=torch.empty_like(q))
+    qp = torch.zeros((1, 2, npad, w.d), dtype=q.dtype, device=dev)
+    wsa = F.alloc_workspace(F.fvattn_workspace_bytes(F.FVATTN_OP_SPARSE_FWD, 1, 2, w.N, w.d, w.block), dev)
+    with pytest.raises(ValueError):      # output of the wrong length
+        F.fvattn_sparse_fwd(qp, qp, qp, torch.empty_like(q), idx, cnt, w.N, w.block, wsa)
+    with pytest.raises(ValueError):      # lse of the wrong length
+        F.fvattn_dense_fwd(qp, qp, qp, torch.empty_like(qp), w.N, w.block, wsa,
+                           lse=torch.empty((1, 2, w.N), dtype=torch.float32, device=dev))
+    with pytest.raises(ValueError):      # x of the wrong length for the grid
+        F.fvattn_permute(qp, torch.empty_like(qp), grid)
+    # the well-formed calls go through
+    F.fvattn_route(q, k, grid, 0.9, 1, idx, cnt, hw, ws)
+    assert F.fvattn_workspace_status(ws) == F.FVATTN_OK

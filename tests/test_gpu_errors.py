@@ -120,3 +120,32 @@ def test_invalid_lists_in_the_fp8v_path_are_reported():
         rows = slice(i * bs, min((i + 1) * bs, w.N))
         mx, _ = attention_errors(op[b, h, rows].float().cpu().numpy(), op_good[b, h, rows].float().cpu().numpy())
         assert mx <= BF16_MAX_ABS, (b, h, i, mx)
+
+
+def test_bounded_waits_run_out_and_report_a_timeout():
+    """The waits every kernel uses, on barriers nothing arrives at: each gives up after
+    the limit, the abort flag releases the second waiter, the status word reads
+    FVATTN_ERR_TIMEOUT, and the context keeps working (no fault, no hang)."""
+    dev = torch.device("cuda")
+    res = torch.full((8,), -1, dtype=torch.int64, device=dev)
+    ws = F.alloc_workspace(256, dev)
+    F.fvattn_wait_selftest(res, ws)
+    assert F.fvattn_workspace_status(ws) == F.FVATTN_ERR_TIMEOUT
+    r = res.cpu().tolist()
+    limit = r[6]
+    assert limit == 2_000_000_000
+    assert r[0] == 0 and limit <= r[1] < limit + 500_000_000, r          # ran out at the limit
+    assert r[2] == 0 and r[3] < limit + 500_000_000, r                   # released, not stuck
+    assert r[4] == 0 and limit <= r[5] < limit + 500_000_000, r          # drain wait bounded too
+    assert r[7] == 1, r                                                  # abort flag raised
+    # the same workspace and context still run a kernel and report OK
+    w = S.Workload("after-timeout", 1, 2, 128, "bf16", (2, 8, 16), (1, 8, 16), 128, 0.9, 1, seed=66)
+    q, k, v = S.make_qkv(w, device=dev)
+    grid = F.Grid.make(w.grid, w.tile, w.block)
+    qp, kp, vp = (torch.empty((w.B, w.H, grid.nb * w.block, w.d), dtype=q.dtype, device=dev) for _ in range(3))
+    for x, y in ((q, qp), (k, kp), (v, vp)):
+        F.fvattn_permute(x, y, grid)
+    op = torch.empty_like(qp)
+    F.fvattn_dense_fwd(qp, kp, vp, op, w.N, w.block, ws)
+    assert F.fvattn_workspace_status(ws) == F.FVATTN_OK
+    assert torch.isfinite(op[:, :, : w.N].float()).all()

@@ -178,7 +178,7 @@ def _select_gpu(w, imp_t, p, k_min):
 @pytest.mark.parametrize("w", [ODD128, BS64], ids=lambda w: w.name)
 @pytest.mark.parametrize("p,k_min", [(0.8, 2), (0.5, 1), (1.0, 1)])
 def test_select_topp_on_importance_matches_oracle(w, p, k_min):
-    from parity import check_lists_valid, compare_masks
+    from parity import assert_mask_parity, check_lists_valid, compare_masks
     q, k, v = S.make_qkv(w, device="cuda")
     grid, qp, kp, _, _, _ = _route_gpu(w, q, k)
     vp = torch.empty_like(qp)
@@ -193,10 +193,9 @@ def test_select_topp_on_importance_matches_oracle(w, p, k_min):
     ocnt = np.empty(scores.shape[:-1], dtype=np.int64)
     for row in np.ndindex(*ocnt.shape):
         order[row], ocnt[row] = O.topp_topk_select(scores[row], p, k_min)
-    n_mis, n_border, hard = compare_masks(mask_from_lists(idx, cnt, nb),
-                                          {"scores": scores, "order": order, "cnt": ocnt}, p)
-    assert not hard, hard[:3]
-    print(f"{w.name} p={p} k_min={k_min}: mismatched={n_mis} borderline={n_border}")
+    assert_mask_parity(compare_masks(mask_from_lists(idx, cnt, nb),
+                                     {"scores": scores, "order": order, "cnt": ocnt}, p),
+                       f"{w.name} p={p} k_min={k_min}")
 
 
 def test_gsrs_search_over_candidates():

@@ -13,8 +13,8 @@ import oracle as O
 import synthetic as S
 from oracle import hilbert_oracle as Hb
 from oracle import lvsa_oracle as L
-from parity import (BF16_MAX_ABS, BF16_MEAN_ABS, attention_errors, check_lists_valid, compare_masks,
-                    mask_from_lists)
+from parity import (BF16_MAX_ABS, BF16_MEAN_ABS, assert_mask_parity, attention_errors, check_lists_valid,
+                    compare_masks, mask_from_lists)
 
 pytestmark = pytest.mark.gpu
 
@@ -64,9 +64,7 @@ def test_permute_and_route_in_hilbert_order(w):
     assert np.array_equal(_np(qp), O.permute(qn, perm, w.block))
     idx, cnt = kv_idx.cpu().numpy(), kv_cnt.cpu().numpy()
     check_lists_valid(idx, cnt, nb, w.k_min)
-    n_mis, n_border, hard = compare_masks(mask_from_lists(idx, cnt, nb), orc, w.p)
-    assert not hard, hard[:5]
-    print(f"{w.name}: mismatched={n_mis} borderline={n_border}")
+    assert_mask_parity(compare_masks(mask_from_lists(idx, cnt, nb), orc, w.p), w.name)
 
 
 def test_lvsa_lists_in_hilbert_order():
