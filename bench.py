@@ -295,10 +295,12 @@ def run_lvsa(F, w, path, stream, warmup, eff_flops_fn):
             "head_work_max_over_mean": float(hwn.max() / hwn.mean()), "_lists": (idx, cnt)}
 
 
-def run_fp8v(F, w, path, stream, warmup, eff):
+def run_fp8v(F, w, path, stream, warmup, eff, q, k, v):
     """Attention with the per-channel E4M3 V (8-bit P.V product) on the routed lists
-    of the timed call: the quantization step, the sparse and dense launches, and the
-    output's distance from the bf16-V launch on the same inputs."""
+    of the timed call: the quantization step (alone, and fused with the permutation),
+    the sparse and dense launches, the output's distance from the bf16-V launch on the
+    same inputs, and the whole step with the E4M3 V (route, fused permutation and
+    quantization of V, attention, inverse permutation)."""
     dev = path.qp.device
     vq = torch.empty(path.vp.shape, dtype=torch.uint8, device=dev)
     vs = torch.empty((w.B, w.H, w.d), dtype=torch.float32, device=dev)
@@ -313,8 +315,23 @@ def run_fp8v(F, w, path, stream, warmup, eff):
     diff = (out8[:, :, :w.N].float() - path.op[:, :, :w.N].float()).abs()
     dense_ms = _median_ms(lambda: F.fvattn_dense_fwd_fp8v(path.qp, path.kp, vq, vs, out8, w.N, w.block,
                                                           path.ws_attn), stream, warmup, 3)
-    if F.fvattn_workspace_status(wsq) != F.FVATTN_OK or F.fvattn_workspace_status(path.ws_attn) != F.FVATTN_OK:
+    fused_ms = _median_ms(lambda: F.fvattn_permute_quantize_v(v, path.grid, vq, vs, wsq), stream, warmup, 5)
+    p8 = F.FVAttnPath(w.B, w.H, w.grid, w.tile, w.block, w.d, torch.bfloat16, w.p, w.k_min, device=dev,
+                      v_format="e4m3")
+
+    def step8():
+        p8.route(q, k)
+        p8.prepare_v(v)
+        p8.attend()
+        F.fvattn_permute(p8.op, p8.out, p8.grid, inverse=True)
+
+    step_ms = _median_ms(step8, stream, warmup, 5)
+    same_codes = bool(torch.equal(p8.vq, vq) and torch.equal(p8.vscale, vs))
+    if F.fvattn_workspace_status(wsq) != F.FVATTN_OK or F.fvattn_workspace_status(path.ws_attn) != F.FVATTN_OK \
+            or F.fvattn_workspace_status(p8.ws_attn) != F.FVATTN_OK or F.fvattn_workspace_status(p8.ws_quant) != F.FVATTN_OK:
         raise RuntimeError("kernel status word set in the FP8 V run")
+    del p8
+    torch.cuda.empty_cache()
     v_bytes = w.B * w.H * w.N * w.d * 2
     q_bytes = w.B * w.H * path.npad * w.d
     d_flops = dense_flops(w.B, w.H, w.N, w.d)
@@ -323,6 +340,13 @@ def run_fp8v(F, w, path, stream, warmup, eff):
             "quantize_gbs": (v_bytes + q_bytes) / (quant_ms * 1e-3) / 1e9,
             "quantize_bytes": {"algorithmic": v_bytes + q_bytes, "moved": 2 * v_bytes + q_bytes,
                                "note": "two passes over V: channel maxima, then encoding"},
+            "permute_quantize_ms": fused_ms,
+            "permute_quantize_gbs": (2 * v_bytes + q_bytes) / (fused_ms * 1e-3) / 1e9,
+            "permute_quantize_note": "fvattn_permute_quantize_v from the raster-order V: reads V twice "
+                                     "(maxima, gather + encode), writes the codes; equal codes to permute + "
+                                     f"quantize: {same_codes}",
+            "step_ms": step_ms,
+            "step_note": "route + fused permutation/quantization of V + sparse attention (E4M3 P.V) + inverse",
             "attention_ms": sparse_ms, "effective_tflops": eff / (sparse_ms * 1e-3) / 1e12,
             "dense_attention_ms": dense_ms, "dense_tflops": d_flops / (dense_ms * 1e-3) / 1e12,
             "max_abs_diff_vs_bf16_v": float(diff.max()), "mean_abs_diff_vs_bf16_v": float(diff.mean())}
@@ -535,8 +559,9 @@ def run_fvattn(args):
                         lvsa_lists=(lvsa.pop("_lists") if lvsa is not None else None))
     fp8v = None
     if not args.no_fp8v:
-        fp8v = run_fp8v(F, w, path, stream, args.warmup, eff)
+        fp8v = run_fp8v(F, w, path, stream, args.warmup, eff, q, k, v)
         fp8v["speedup_vs_bf16_v"] = ms_attn / fp8v["attention_ms"]
+        fp8v["step_speedup_vs_bf16_step"] = ms_step / fp8v["step_ms"]
         fp8v["dense_speedup_vs_bf16_v"] = ms_dense / fp8v["dense_attention_ms"]
 
     # ---- e2e through the public API with pinned host buffers: every step uploads its

@@ -61,7 +61,8 @@ EXPORTED = ("fvattn_workspace_bytes", "fvattn_permute", "fvattn_route", "fvattn_
             "fvattn_sparse_fwd", "fvattn_dense_fwd", "fvattn_block_importance", "fvattn_attention_recall",
             "fvattn_select_topp", "fvattn_lvsa_lists", "fvattn_hilbert_table", "fvattn_quantize_v",
             "fvattn_sparse_fwd_fp8v", "fvattn_dense_fwd_fp8v",
-            "fvattn_workspace_status", "fvattn_status_string", "fvattn_wait_selftest")
+            "fvattn_workspace_status", "fvattn_status_string", "fvattn_wait_selftest",
+            "fvattn_permute_quantize_v")
 
 
 class Grid(ctypes.Structure):
@@ -113,6 +114,9 @@ _lib.fvattn_dense_fwd.restype = _c_int
 _lib.fvattn_quantize_v.argtypes = [_c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_void_p, _c_void_p,
                                    _c_void_p, _c_size_t, _c_void_p]
 _lib.fvattn_quantize_v.restype = _c_int
+_lib.fvattn_permute_quantize_v.argtypes = [_c_void_p, _c_int, _c_int, _c_int, _c_int, ctypes.POINTER(Grid),
+                                           _c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_void_p]
+_lib.fvattn_permute_quantize_v.restype = _c_int
 _lib.fvattn_sparse_fwd_fp8v.argtypes = [_c_void_p] * 9 + [_c_int] * 5 + [_c_float, _c_void_p, _c_size_t,
                                                                       _c_void_p]
 _lib.fvattn_sparse_fwd_fp8v.restype = _c_int
@@ -356,6 +360,26 @@ def fvattn_quantize_v(vp, vq, vscale, N: int, block: int, workspace, stream=None
     return vq, vscale
 
 
+def fvattn_permute_quantize_v(v, grid: Grid, vq, vscale, workspace, stream=None):
+    """Raster-order V [B,H,N,128] bf16 -> E4M3 codes vq [B,H,Npad,128] uint8 in the grid's
+    block order and scales vscale [B,H,128] fp32 (the permutation and the quantization
+    in one pass over the codes)."""
+    _need_cuda(v, vq, vscale, workspace)
+    dev = v.device
+    B, H, N, d = v.shape
+    if v.dtype != torch.bfloat16:
+        raise TypeError("v must be bf16")
+    if N != grid.N:
+        raise ValueError(f"v has {N} tokens, the grid {grid.N}")
+    _expect(vq, "vq", dev, (B, H, grid.nb * grid.block, d), torch.uint8)
+    _expect(vscale, "vscale", dev, (B, H, d), torch.float32)
+    _expect_ws(workspace, dev)
+    _check(_call(dev, _lib.fvattn_permute_quantize_v, _ptr(v), B, H, N, d, ctypes.byref(grid), _ptr(vq),
+                 _ptr(vscale), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                 _stream(stream, dev)), "fvattn_permute_quantize_v")
+    return vq, vscale
+
+
 def fvattn_sparse_fwd_fp8v(qp, kp, vq, vscale, out, kv_idx, kv_cnt, N: int, block: int, workspace,
                            scale=None, lse=None, block_lse=None, stream=None):
     """fvattn_sparse_fwd with the E4M3 V of fvattn_quantize_v (8-bit P.V product)."""
@@ -508,8 +532,9 @@ class FVAttnPath:
     also permutes q and k), permute v, block-sparse attention, inverse permute.
     ``dense=True`` runs the dense kernel instead of routing. ``order="hilbert"``
     orders blocks along the Hilbert curve (the table is built once here) instead
-    of 3-D tiles. ``v_format="e4m3"`` quantizes the permuted V per channel
-    (fvattn_quantize_v) and runs attention with the 8-bit P.V product.
+    of 3-D tiles. ``v_format="e4m3"`` permutes and quantizes V per channel in one
+    call (fvattn_permute_quantize_v; no bf16 permuted V is formed) and runs
+    attention with the 8-bit P.V product.
     """
 
     def __init__(self, B, H, grid, tile, block, d, dtype, p, k_min, device="cuda", order="tiles",
@@ -536,7 +561,7 @@ class FVAttnPath:
         shp = (B, H, self.npad, d)
         self.qp = torch.empty(shp, dtype=dtype, device=dev)
         self.kp = torch.empty(shp, dtype=dtype, device=dev)
-        self.vp = torch.empty(shp, dtype=dtype, device=dev)
+        self.vp = None if self.fp8v else torch.empty(shp, dtype=dtype, device=dev)
         self.op = torch.empty(shp, dtype=dtype, device=dev)
         self.out = torch.empty((B, H, self.N, d), dtype=dtype, device=dev)
         self.kv_idx = torch.empty((B, H, self.nb, self.nb), dtype=torch.int32, device=dev)
@@ -573,9 +598,19 @@ class FVAttnPath:
         fvattn_route(q, k, self.grid, self.p, self.k_min, self.kv_idx, self.kv_cnt,
                      self.head_work, self.ws_route, qp_out=self.qp, kp_out=self.kp)
 
-    def attend(self, dense=False):
+    def prepare_v(self, v):
+        """V [B,H,N,d] (original order) into the attention kernel's input: the permuted
+        bf16 V, or (E4M3 path) the permuted per-channel E4M3 codes and scales, formed
+        from the raster-order V in one fused call."""
         if self.fp8v:
-            fvattn_quantize_v(self.vp, self.vq, self.vscale, self.N, self.block, self.ws_quant)
+            fvattn_permute_quantize_v(v, self.grid, self.vq, self.vscale, self.ws_quant)
+        else:
+            fvattn_permute(v, self.vp, self.grid)
+
+    def attend(self, dense=False):
+        """Attention over the prepared inputs (qp, kp from route or permute; V from
+        prepare_v)."""
+        if self.fp8v:
             if dense:
                 fvattn_dense_fwd_fp8v(self.qp, self.kp, self.vq, self.vscale, self.op, self.N, self.block,
                                       self.ws_attn)
@@ -596,7 +631,7 @@ class FVAttnPath:
             fvattn_permute(k, self.kp, self.grid)
         else:
             self.route(q, k)
-        fvattn_permute(v, self.vp, self.grid)
+        self.prepare_v(v)
         self.attend(dense=dense)
         dst = self.out if out is None else out
         fvattn_permute(self.op, dst, self.grid, inverse=True)

@@ -46,6 +46,8 @@ cudaError_t launch_quantize_v(const void* v, int BH, int N, int npad, uint8_t* v
                               unsigned int* amax_bits, cudaStream_t st);
 size_t vquant_ws_bytes(int BH);
 cudaError_t launch_wait_selftest(long long* out, int* status, cudaStream_t st);
+cudaError_t launch_permute_quantize_v(const void* v, int BH, int N, int bs, const TileGeom& g, uint8_t* vq,
+                                      float* vscale, unsigned int* amax_bits, cudaStream_t st);
 int hilbert_bits(int extent);
 int next_pow2(int n);
 }  // namespace fvattn
@@ -382,6 +384,30 @@ fvattn_status fvattn_quantize_v(const void* vp, int B, int H, int N, int d, int 
   return from_cuda(fvattn::launch_quantize_v(vp, B * H, N, static_cast<int>(npad), vq, vscale,
                                              reinterpret_cast<unsigned int*>(base + kWsHeaderBytes),
                                              st));
+}
+
+fvattn_status fvattn_permute_quantize_v(const void* v, int B, int H, int N, int d, const fvattn_grid* grid,
+                                        uint8_t* vq, float* vscale, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+  if (!v || !vq || !vscale) return FVATTN_ERR_INVALID_ARG;
+  if (!aligned(v, 16) || !aligned(vq, 16) || !aligned(vscale, 16)) return FVATTN_ERR_INVALID_ARG;
+  if (!valid_grid(grid, N) || !valid_sizes(B, H, N, d, grid->block)) return FVATTN_ERR_INVALID_ARG;
+  if (d != 128) return FVATTN_ERR_UNSUPPORTED;
+  const int block = grid->block;
+  const size_t npad = static_cast<size_t>(num_blocks(N, block)) * block;
+  const size_t bh = static_cast<size_t>(B) * H;
+  if (ranges_overlap(v, bh * N * d * 2, vq, bh * npad * d) ||
+      ranges_overlap(v, bh * N * d * 2, vscale, bh * d * 4) ||
+      ranges_overlap(vq, bh * npad * d, vscale, bh * d * 4))
+    return FVATTN_ERR_INVALID_ARG;
+  const size_t need = fvattn_workspace_bytes(FVATTN_OP_QUANT_V, B, H, N, d, block);
+  const fvattn_status wst = check_ws(workspace, workspace_bytes, need);
+  if (wst != FVATTN_OK) return wst;
+  auto st = static_cast<cudaStream_t>(stream);
+  auto base = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(base, 0, need, st) != cudaSuccess) return FVATTN_ERR_CUDA;
+  return from_cuda(fvattn::launch_permute_quantize_v(v, B * H, N, block, geom_of(grid), vq, vscale,
+                                                     reinterpret_cast<unsigned int*>(base + kWsHeaderBytes), st));
 }
 
 fvattn_status fvattn_sparse_fwd_fp8v(const void* qp, const void* kp, const uint8_t* vq,

@@ -13,8 +13,8 @@
 //   - At most kScratchBytes (96 MiB) of scratch: sizes whose route workspace
 //     (fvattn_workspace_bytes(FVATTN_OP_ROUTE, ...)) is larger are rejected with
 //     FVATTN_ERR_WORKSPACE before anything is launched. The Wan-14B 720p shape
-//     (40 heads, 591 blocks, d = 128) needs 80.1 MB (block means 24.2 MB, block
-//     scores 55.9 MB) and fits.
+//     (40 heads, 591 blocks, d = 128) needs 80.2 MB (block means 24.2 MB, block
+//     scores 56.0 MB) and fits.
 //   - Every call on a device uses the same array and leaves its contents for
 //     the next call. The router clears the status word at the start of each
 //     call and overwrites the block means and scores completely, so no stale value is

@@ -19,6 +19,13 @@
 // memory and merged with an integer atomicMax on the float bits (exact for
 // values >= 0); (2) the encoding, same thread mapping, 8 bytes stored per
 // thread. Both read V rows as 16-byte vectors, so a warp covers two full rows.
+//
+// Fused with the block-order permutation (launch_permute_quantize_v): the
+// maxima do not depend on the token order, so pass (1) reads V in raster order,
+// and pass (2) gathers each block's rows from raster order (as the permutation
+// does) and encodes them, so V is read twice and the codes written once; the
+// permuted bf16 V is never formed. Its codes and scales equal those of the
+// permutation followed by the quantization, bit for bit.
 #include "common.cuh"
 
 namespace fvattn {
@@ -111,6 +118,64 @@ __global__ void __launch_bounds__(kQuantThreads)
   }
 }
 
+// One CTA per (block of bs permuted rows, head): the rows' raster sources, then
+// the encoding of each source row into its permuted position (pad rows 0).
+__global__ void __launch_bounds__(kQuantThreads)
+    vquant_gather_encode_kernel(const uint4* __restrict__ v, int N, int nb, int bs, TileGeom g,
+                                const unsigned int* __restrict__ amax_bits, uint2* __restrict__ vq,
+                                float* __restrict__ vscale) {
+  __shared__ int src[128];
+  const int i = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int cg = threadIdx.x & 15;
+  const int r0 = threadIdx.x >> 4;
+  for (int r = threadIdx.x; r < bs; r += blockDim.x) {
+    const int pos = i * bs + r;
+    src[r] = pos < N ? source_index(pos, N, g) : -1;
+  }
+  const unsigned int* am = amax_bits + static_cast<size_t>(bh) * kQuantD;
+  float inv[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float a = __uint_as_float(__ldg(am + cg * 8 + k));
+    inv[k] = a >= kAmaxZero ? __fdiv_rn(kE4M3Max, a) : 0.f;
+  }
+  if (i == 0 && threadIdx.x < kQuantD) {
+    const float a = __uint_as_float(__ldg(am + threadIdx.x));
+    vscale[static_cast<size_t>(bh) * kQuantD + threadIdx.x] = a >= kAmaxZero ? __fdiv_rn(a, kE4M3Max) : 0.f;
+  }
+  __syncthreads();
+  const uint4* base = v + static_cast<size_t>(bh) * N * (kQuantD / 8);
+  uint2* out = vq + (static_cast<size_t>(bh) * nb * bs + static_cast<size_t>(i) * bs) * (kQuantD / 8);
+  constexpr int kRowsPerPass = kQuantThreads / 16;
+  constexpr int kInflight = 8;
+  for (int rb = 0; rb < bs; rb += kRowsPerPass * kInflight) {
+    uint4 x[kInflight];
+#pragma unroll
+    for (int k = 0; k < kInflight; ++k) {
+      const int r = rb + r0 + k * kRowsPerPass;
+      const int s = r < bs ? src[r] : -1;
+      x[k] = s >= 0 ? __ldg(base + static_cast<size_t>(s) * (kQuantD / 8) + cg) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int k = 0; k < kInflight; ++k) {
+      const int r = rb + r0 + k * kRowsPerPass;
+      if (r >= bs) continue;
+      uint2 w = make_uint2(0u, 0u);
+      if (src[r] >= 0) {
+        float f[8];
+        bf16x8_to_float(x[k], f);
+        uint32_t h[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          h[e] = cvt_e4m3x2(__fmul_rn(f[2 * e], inv[2 * e]), __fmul_rn(f[2 * e + 1], inv[2 * e + 1]));
+        w = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+      }
+      out[static_cast<size_t>(r) * (kQuantD / 8) + cg] = w;
+    }
+  }
+}
+
 size_t vquant_ws_bytes(int BH) { return static_cast<size_t>(BH) * kQuantD * sizeof(unsigned int); }
 
 // amax_bits must hold vquant_ws_bytes(BH) zeroed bytes (the caller clears them
@@ -124,6 +189,21 @@ cudaError_t launch_quantize_v(const void* v, int BH, int N, int npad, uint8_t* v
   const dim3 ge((npad + kQuantRows - 1) / kQuantRows, BH);
   vquant_encode_kernel<<<ge, kQuantThreads, 0, st>>>(static_cast<const uint4*>(v), N, npad, amax_bits,
                                                      reinterpret_cast<uint2*>(vq), vscale);
+  return cudaGetLastError();
+}
+
+// V in raster order [BH, N, 128] bf16 -> codes in the block order of g
+// [BH, nb*bs, 128] and scales; amax_bits as above.
+cudaError_t launch_permute_quantize_v(const void* v, int BH, int N, int bs, const TileGeom& g, uint8_t* vq,
+                                      float* vscale, unsigned int* amax_bits, cudaStream_t st) {
+  const int nb = (N + bs - 1) / bs;
+  const dim3 ga((N + kQuantRows - 1) / kQuantRows, BH);
+  vquant_amax_kernel<<<ga, kQuantThreads, 0, st>>>(static_cast<const uint4*>(v), N, N, amax_bits);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const dim3 ge(nb, BH);
+  vquant_gather_encode_kernel<<<ge, kQuantThreads, 0, st>>>(static_cast<const uint4*>(v), N, nb, bs, g, amax_bits,
+                                                            reinterpret_cast<uint2*>(vq), vscale);
   return cudaGetLastError();
 }
 

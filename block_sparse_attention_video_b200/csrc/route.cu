@@ -3,23 +3,28 @@
 //
 // Two kernels, each at high occupancy:
 //   1. block_scores_kernel: S[b,h,i,j] = scale * qbar_i . kbar_j for every pair
-//      of blocks, fp32, as a 64 x 64 tiled SIMT product (4 x 4 outputs per
-//      thread, both tiles staged k-major in shared memory); S goes to the route
-//      workspace.
-//   2. select_rows_kernel: one warp per (b, h, query block) row, the row staged
-//      in shared memory: max-subtracted softmax (expf, fixed-order warp sums),
+//      of blocks, fp32, as a 128 x 128 tiled SIMT product (8 x 8 outputs per
+//      thread from register-held operands, d staged 32 at a time k-major in
+//      shared memory); S goes to the route workspace with its row stride padded
+//      to a multiple of 4 so that every thread stores whole float4s.
+//   2. select_rows_kernel: one warp per (b, h, query block) row, the row held in
+//      registers (32 per lane and up to 48 values per lane; longer rows are staged
+//      in shared memory): max-subtracted softmax (expf, fixed-order warp sums),
 //      then the Top-p cut found without sorting: the largest value v* with
-//      F(v*) = sum_{s_j >= v*} s_j >= p, located by bisection on the bit
-//      pattern of non-negative floats (the computed F is monotone in v because
-//      fp32 sums of non-negative terms are monotone in each term); ties at v*
-//      are taken in block-index order until the sum reaches p. F only changes at
-//      the row's values, so v* is one of them: the bisection also counts the
-//      values at or above each bound and stops as soon as one distinct value is
-//      left between them, which is then v*. If the Top-k floor is larger, the
-//      k_min-th largest value is found the same way on counts. The selected
-//      blocks are compacted in ascending index order with warp ballots, the
-//      count is stored and added to the per-head work.
-// Deterministic: every sum has a fixed order.
+//      F(v*) = sum_{s_j >= v*} s_j >= p. F is evaluated with each lane's fp32
+//      partial sum (fixed order) rounded to a 2^-31 fixed point and added
+//      exactly with one integer warp reduction, so the computed F is monotone in
+//      v and deterministic. v* is located by a search on the bit pattern of
+//      non-negative floats between the row's smallest and largest value, that
+//      alternates interpolation on F with plain bisection (the interpolation
+//      usually lands near the cut, the bisection bounds the worst case); each
+//      step also counts the values at or above the probe and the search stops as
+//      soon as one distinct value is left in the bracket, which is then v*. Ties
+//      at v* are taken in block-index order until the sum reaches p. If the Top-k
+//      floor is larger, the k_min-th largest value is found the same way on
+//      counts. The selected blocks are compacted in ascending index order with
+//      warp ballots, the count is stored and added to the per-head work.
+// Deterministic: every sum has a fixed order or is an exact integer sum.
 #include <cfloat>
 
 #include "common.cuh"
@@ -44,67 +49,114 @@ __device__ __forceinline__ int warp_sum_int(int v) {
   return v;
 }
 
-// F(thr) = sum of s_j >= thr, same association order for every thr.
-__device__ __forceinline__ float mass_at_least(const float* s, int nb, float thr, int lane) {
-  float a = 0.f;
-  for (int j = lane; j < nb; j += 32) {
-    const float v = s[j];
-    a += v >= thr ? v : 0.f;
+constexpr float kFix = 2147483648.0f;   // 2^31: masses in [0, 1] as 2^-31 fixed point
+
+// Fixed-point mass of one lane's fp32 partial sum (at most 1 + rounding).
+__device__ __forceinline__ uint32_t to_fix(float a) { return __float2uint_rn(a * kFix); }
+
+// Probe of the search: interpolation of F between the bracket's ends on odd
+// steps, bisection of the bit range on even steps; always strictly inside
+// (lo, hi). lo, hi are bit patterns of non-negative floats, hi - lo > 1.
+__device__ __forceinline__ uint32_t probe(uint32_t lo, uint32_t hi, uint32_t f_lo, uint32_t f_hi,
+                                          uint32_t target, int step) {
+  uint32_t mid = lo + ((hi - lo) >> 1);
+  if ((step & 1) && f_lo > f_hi) {
+    const float vl = __uint_as_float(lo), vh = __uint_as_float(hi);
+    const float t = static_cast<float>(f_lo - target) / static_cast<float>(f_lo - f_hi);
+    const uint32_t m = __float_as_uint(fmaf(vh - vl, t, vl));
+    mid = min(max(m, lo + 1u), hi - 1u);
   }
-  return warp_sum(a);
+  return mid;
 }
 
-__device__ __forceinline__ int count_at_least(const float* s, int nb, float thr, int lane) {
-  unsigned c = 0u;
-  for (int j = lane; j < nb; j += 32) c += s[j] >= thr ? 1u : 0u;
-  return static_cast<int>(__reduce_add_sync(0xffffffffu, c));
-}
-
-// The only value of the row in [lo, hi) (the caller knows there is exactly one).
-__device__ __forceinline__ uint32_t only_value_below(const float* s, int nb, uint32_t hi, int lane) {
-  unsigned m = 0u;
-  for (int j = lane; j < nb; j += 32) {
-    const unsigned b = __float_as_uint(s[j]);
-    if (b < hi) m = max(m, b);
+// One row of up to 32 * VPL values held in registers, value t of a lane being
+// element t * 32 + lane. Elements past nb hold -1 (never selected: every
+// threshold is a non-negative float).
+template <int VPL>
+__device__ void select_row_reg(const float* __restrict__ src, int nb, float p, int k_min,
+                               int* __restrict__ out_idx, int* __restrict__ out_cnt,
+                               unsigned long long* head_work, int* status, int lane, bool softmax) {
+  float v[VPL];
+#pragma unroll
+  for (int t = 0; t < VPL; ++t) {
+    const int j = t * 32 + lane;
+    v[t] = j < nb ? src[j] : -INFINITY;
   }
-  return __reduce_max_sync(0xffffffffu, m);
-}
-
-// One importance row (already scaled logits in s[0..nb)), one warp.
-// With softmax == false the row already holds importances (non-negative,
-// summing to one over the evaluated blocks) and goes straight to selection.
-__device__ void select_row(float* s, int nb, float p, int k_min, int* __restrict__ out_idx,
-                           int* __restrict__ out_cnt, unsigned long long* head_work,
-                           int* status, int lane, bool softmax) {
   if (softmax) {
-    // softmax over the row, max subtracted
+    // softmax over the row, max subtracted; pads (-inf) give 0 and are then set to -1
     float m = -FLT_MAX;
-    for (int j = lane; j < nb; j += 32) m = fmaxf(m, s[j]);
+#pragma unroll
+    for (int t = 0; t < VPL; ++t) m = fmaxf(m, v[t]);
     m = warp_max(m);
     float z = 0.f;
-    for (int j = lane; j < nb; j += 32) {
-      const float e = expf(s[j] - m);
-      s[j] = e;
-      z += e;
+#pragma unroll
+    for (int t = 0; t < VPL; ++t) {
+      v[t] = expf(v[t] - m);
+      z += v[t];
     }
     z = warp_sum(z);
-    for (int j = lane; j < nb; j += 32) s[j] = s[j] / z;
+    const float rz = 1.0f / z;
+#pragma unroll
+    for (int t = 0; t < VPL; ++t) v[t] = t * 32 + lane < nb ? v[t] * rz : -1.f;
   } else {
     // negative or non-finite importances are invalid input: clamped to 0, recorded
     bool bad = false;
-    for (int j = lane; j < nb; j += 32) {
-      const float v = s[j];
-      if (!(v >= 0.f && v <= 1.f)) {
-        s[j] = v > 1.f ? 1.f : 0.f;
+#pragma unroll
+    for (int t = 0; t < VPL; ++t) {
+      if (t * 32 + lane >= nb) {
+        v[t] = -1.f;
+      } else if (!(v[t] >= 0.f && v[t] <= 1.f)) {
+        v[t] = v[t] > 1.f ? 1.f : 0.f;
         bad = true;
       }
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) record_status(status, FVATTN_ERR_INVALID_ARG);
   }
-  __syncwarp();
+
+  // F(x) in fixed point and the number of values >= x, one pass over the row
+  auto mass_count = [&](float x, uint32_t& F, int& C) {
+    float a = 0.f;
+    unsigned c = 0u;
+#pragma unroll
+    for (int t = 0; t < VPL; ++t) {
+      const bool ge = v[t] >= x;
+      a += ge ? v[t] : 0.f;
+      c += ge ? 1u : 0u;
+    }
+    F = __reduce_add_sync(0xffffffffu, to_fix(a));
+    C = static_cast<int>(__reduce_add_sync(0xffffffffu, c));
+  };
+  auto count_ge = [&](float x) -> int {
+    unsigned c = 0u;
+#pragma unroll
+    for (int t = 0; t < VPL; ++t) c += v[t] >= x ? 1u : 0u;
+    return static_cast<int>(__reduce_add_sync(0xffffffffu, c));
+  };
+  // the only value in [lo, hi) when the caller knows there is exactly one (pads,
+  // negative, compare above every bit pattern of a non-negative float)
+  auto only_below = [&](uint32_t hi) -> uint32_t {
+    unsigned m = 0u;
+#pragma unroll
+    for (int t = 0; t < VPL; ++t) {
+      const unsigned bits = __float_as_uint(v[t]);
+      if (bits < hi) m = max(m, bits);
+    }
+    return __reduce_max_sync(0xffffffffu, m);
+  };
+  // bracket of the valid values: smallest and largest (as bit patterns)
+  unsigned vmin = 0x7F800000u, vmax = 0u;
+#pragma unroll
+  for (int t = 0; t < VPL; ++t) {
+    if (v[t] >= 0.f) {
+      vmin = min(vmin, __float_as_uint(v[t]));
+      vmax = max(vmax, __float_as_uint(v[t]));
+    }
+  }
+  vmin = __reduce_min_sync(0xffffffffu, vmin);
+  vmax = __reduce_max_sync(0xffffffffu, vmax);
 
   int cnt;
-  float thr;      // selected: s > thr, plus the first take_eq entries equal to thr
+  float thr;      // selected: v > thr, plus the first take_eq entries equal to thr
   int take_eq;
   if (p >= 1.f || k_min >= nb) {
     cnt = nb;
@@ -114,35 +166,36 @@ __device__ void select_row(float* s, int nb, float p, int k_min, int* __restrict
     int n_p;
     float vstar = 0.f;
     int cgt = 0;
-    const float total = mass_at_least(s, nb, 0.f, lane);
-    if (total < p) {
+    const uint32_t target = to_fix(p);
+    uint32_t total;
+    int call;
+    mass_count(0.f, total, call);
+    if (total < target) {
       n_p = nb;
     } else {
-      uint32_t lo = 0u, hi = 0x3F800001u;          // F(lo) >= p > F(hi)
+      uint32_t lo = vmin, hi = vmax + 1u;          // F(lo) >= target > F(hi)
+      uint32_t f_lo = total, f_hi = 0u;
       int c_lo = nb, c_hi = 0;                     // values at or above lo, hi
-      while (hi - lo > 1u && c_lo - c_hi > 1) {
-        const uint32_t mid = lo + ((hi - lo) >> 1);
-        const float fm = mass_at_least(s, nb, __uint_as_float(mid), lane);
-        const int cm = count_at_least(s, nb, __uint_as_float(mid), lane);
-        if (fm >= p) { lo = mid; c_lo = cm; } else { hi = mid; c_hi = cm; }
+      for (int step = 1; hi - lo > 1u && c_lo - c_hi > 1; ++step) {
+        const uint32_t mid = probe(lo, hi, f_lo, f_hi, target, step);
+        uint32_t fm;
+        int cm;
+        mass_count(__uint_as_float(mid), fm, cm);
+        if (fm >= target) { lo = mid; f_lo = fm; c_lo = cm; } else { hi = mid; f_hi = fm; c_hi = cm; }
       }
-      // One value left in [lo, hi): it is v*. (Otherwise lo and hi are adjacent
-      // floats and v* = lo.)
-      if (c_lo - c_hi == 1) lo = only_value_below(s, nb, hi, lane);
+      // F(lo) > F(hi), so [lo, hi) holds at least one value. Either exactly one
+      // is left, which is v*, or lo and hi are adjacent floats and every value
+      // in the bracket equals lo = v*. Either way the values above v* are those
+      // at or above hi: their mass and count are f_hi and c_hi, and the
+      // c_lo - c_hi values equal to v* are taken in index order until p is reached.
+      if (c_lo - c_hi == 1) lo = only_below(hi);
       vstar = __uint_as_float(lo);
-      float sgt = 0.f;
-      int ceq = 0;
-      for (int j = lane; j < nb; j += 32) {
-        const float v = s[j];
-        if (v > vstar) { sgt += v; ++cgt; }
-        ceq += v == vstar ? 1 : 0;
-      }
-      sgt = warp_sum(sgt);
-      cgt = warp_sum_int(cgt);
-      ceq = warp_sum_int(ceq);
+      cgt = c_hi;
+      const int ceq = c_lo - c_hi;
+      const uint32_t fstar = to_fix(vstar);
       int need = 1;
-      float acc = sgt + vstar;
-      while (acc < p && need < ceq) { acc += vstar; ++need; }
+      uint32_t acc = f_hi + fstar;
+      while (acc < target && need < ceq) { acc += fstar; ++need; }
       n_p = cgt + need;
     }
     cnt = min(nb, max(n_p, k_min));
@@ -153,31 +206,31 @@ __device__ void select_row(float* s, int nb, float p, int k_min, int* __restrict
       thr = vstar;
       take_eq = cnt - cgt;
     } else {
-      uint32_t lo = 0u, hi = 0x3F800001u;          // count(lo) >= cnt > count(hi)
+      uint32_t lo = vmin, hi = vmax + 1u;          // count(lo) >= cnt > count(hi)
       int c_lo = nb, c_hi = 0;
       while (hi - lo > 1u && c_lo - c_hi > 1) {
         const uint32_t mid = lo + ((hi - lo) >> 1);
-        const int cm = count_at_least(s, nb, __uint_as_float(mid), lane);
+        const int cm = count_ge(__uint_as_float(mid));
         if (cm >= cnt) { lo = mid; c_lo = cm; } else { hi = mid; c_hi = cm; }
       }
-      if (c_lo - c_hi == 1) lo = only_value_below(s, nb, hi, lane);
+      // as above: the values above the threshold are the c_hi at or above hi
+      if (c_lo - c_hi == 1) lo = only_below(hi);
       thr = __uint_as_float(lo);
-      int gt = 0;
-      for (int j = lane; j < nb; j += 32) gt += s[j] > thr ? 1 : 0;
-      take_eq = cnt - warp_sum_int(gt);
+      take_eq = cnt - c_hi;
     }
   }
 
   // compaction in ascending block index
   const unsigned lt_mask = (1u << lane) - 1u;
   int written = 0, eq_seen = 0;
-  for (int base = 0; base < nb; base += 32) {
-    const int j = base + lane;
-    const float v = j < nb ? s[j] : -2.f;
-    const bool eq = v == thr;
+#pragma unroll
+  for (int t = 0; t < VPL; ++t) {
+    const int j = t * 32 + lane;
+    const bool valid = j < nb;
+    const bool eq = valid && v[t] == thr;
     const unsigned eqb = __ballot_sync(0xffffffffu, eq);
     const int eq_rank = eq_seen + __popc(eqb & lt_mask);
-    const bool sel = v > thr || (eq && eq_rank < take_eq);
+    const bool sel = valid && (v[t] > thr || (eq && eq_rank < take_eq));
     const unsigned sb = __ballot_sync(0xffffffffu, sel);
     if (sel) out_idx[written + __popc(sb & lt_mask)] = j;
     written += __popc(sb);
@@ -190,124 +243,154 @@ __device__ void select_row(float* s, int nb, float p, int k_min, int* __restrict
   }
 }
 
-constexpr int kTile = 64;        // score tile: 64 query blocks x 64 key blocks
-constexpr int kTilePad = kTile + 4;
+constexpr int kTileN = 128;      // score tile: 16*TM query blocks x 128 key blocks
+constexpr int kKc = 32;          // d staged 32 at a time
+constexpr int kTilePad = kTileN + 4;
+#ifndef FVATTN_SCORE_TM
+#define FVATTN_SCORE_TM 8
+#endif
+constexpr int kScoreTM = FVATTN_SCORE_TM;   // query blocks per thread (4 or 8)
 
-// S tile = scale * Qtile . Ktile^T over d; 16 x 16 threads, 4 x 4 outputs each.
-__global__ void __launch_bounds__(kRouteThreads)
+// Row stride of the block score matrix: nb padded to a multiple of 4 floats.
+__host__ __device__ __forceinline__ int scores_ld(int nb) { return (nb + 3) & ~3; }
+
+// S tile = scale * Qtile . Ktile^T over d; 16 x 16 threads, each TM x 8 outputs:
+// rows ty*4 + {0..3} (and 64 + ty*4 + {0..3} when TM = 8), columns tx*4 + {0..3}
+// and 64 + tx*4 + {0..3}, so that a warp's shared-memory reads of a k-slice are
+// contiguous 256-byte runs. Means past nb are read as zero; their (finite)
+// scores land in rows past nb, which are not stored, or in columns past nb,
+// which the selection never reads.
+template <int TM>
+__global__ void __launch_bounds__(kRouteThreads, TM == 8 ? 2 : 3)
     block_scores_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar, int nb, int d,
                         float scale, float* __restrict__ S) {
-  extern __shared__ float4 smem_f4[];
-  float* qs = reinterpret_cast<float*>(smem_f4);   // [d][kTilePad], k-major
-  float* ks = qs + d * kTilePad;                   // [d][kTilePad]
+  constexpr int kTileM = 16 * TM;
+  __shared__ __align__(16) float qs[kKc][kTileM + 4];
+  __shared__ __align__(16) float ks[kKc][kTilePad];
   const int bh = blockIdx.z;
-  const int i0 = blockIdx.y * kTile, j0 = blockIdx.x * kTile;
+  const int i0 = blockIdx.y * kTileM, j0 = blockIdx.x * kTileN;
   const float* qb = qbar + static_cast<size_t>(bh) * nb * d;
   const float* kb = kbar + static_cast<size_t>(bh) * nb * d;
-  const int d4 = d >> 2;
-  // rows of the tile are the fastest index so that the transposing stores hit distinct banks
-  for (int e = threadIdx.x; e < kTile * d4; e += kRouteThreads) {
-    const int r = e % kTile, c = (e / kTile) * 4;
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-    if (i0 + r < nb) a = *reinterpret_cast<const float4*>(qb + static_cast<size_t>(i0 + r) * d + c);
-    if (j0 + r < nb) b = *reinterpret_cast<const float4*>(kb + static_cast<size_t>(j0 + r) * d + c);
-    qs[(c + 0) * kTilePad + r] = a.x;
-    qs[(c + 1) * kTilePad + r] = a.y;
-    qs[(c + 2) * kTilePad + r] = a.z;
-    qs[(c + 3) * kTilePad + r] = a.w;
-    ks[(c + 0) * kTilePad + r] = b.x;
-    ks[(c + 1) * kTilePad + r] = b.y;
-    ks[(c + 2) * kTilePad + r] = b.z;
-    ks[(c + 3) * kTilePad + r] = b.w;
-  }
-  __syncthreads();
+  const int ld = scores_ld(nb);
   const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-  float acc[4][4];
+  float acc[TM][8];
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < TM; ++a)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
+    for (int c = 0; c < 8; ++c) acc[a][c] = 0.f;
+  for (int k0 = 0; k0 < d; k0 += kKc) {
+    // rows of the tile are the fastest index so that the transposing stores hit distinct banks
+    for (int e = threadIdx.x; e < kTileN * (kKc / 4); e += kRouteThreads) {
+      const int r = e % kTileN, cl = (e / kTileN) * 4, c = k0 + cl;
+      float4 ka = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j0 + r < nb) ka = *reinterpret_cast<const float4*>(kb + static_cast<size_t>(j0 + r) * d + c);
+      ks[cl + 0][r] = ka.x;
+      ks[cl + 1][r] = ka.y;
+      ks[cl + 2][r] = ka.z;
+      ks[cl + 3][r] = ka.w;
+      if (r < kTileM) {
+        float4 qa = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i0 + r < nb) qa = *reinterpret_cast<const float4*>(qb + static_cast<size_t>(i0 + r) * d + c);
+        qs[cl + 0][r] = qa.x;
+        qs[cl + 1][r] = qa.y;
+        qs[cl + 2][r] = qa.z;
+        qs[cl + 3][r] = qa.w;
+      }
+    }
+    __syncthreads();
 #pragma unroll 4
-  for (int kk = 0; kk < d; ++kk) {
-    const float4 qa = *reinterpret_cast<const float4*>(qs + kk * kTilePad + ty * 4);
-    const float4 kv = *reinterpret_cast<const float4*>(ks + kk * kTilePad + tx * 4);
-    const float qv[4] = {qa.x, qa.y, qa.z, qa.w};
-    const float kf[4] = {kv.x, kv.y, kv.z, kv.w};
+    for (int kk = 0; kk < kKc; ++kk) {
+      float qv[TM];
+      const float4 q0 = *reinterpret_cast<const float4*>(&qs[kk][ty * 4]);
+      qv[0] = q0.x; qv[1] = q0.y; qv[2] = q0.z; qv[3] = q0.w;
+      if constexpr (TM == 8) {
+        const float4 q1 = *reinterpret_cast<const float4*>(&qs[kk][64 + ty * 4]);
+        qv[4] = q1.x; qv[5] = q1.y; qv[6] = q1.z; qv[7] = q1.w;
+      }
+      const float4 k0v = *reinterpret_cast<const float4*>(&ks[kk][tx * 4]);
+      const float4 k1v = *reinterpret_cast<const float4*>(&ks[kk][64 + tx * 4]);
+      const float kf[8] = {k0v.x, k0v.y, k0v.z, k0v.w, k1v.x, k1v.y, k1v.z, k1v.w};
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+      for (int a = 0; a < TM; ++a)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(qv[a], kf[c], acc[a][c]);
+        for (int c = 0; c < 8; ++c) acc[a][c] = fmaf(qv[a], kf[c], acc[a][c]);
+    }
+    __syncthreads();
   }
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int i = i0 + ty * 4 + a;
-    if (i >= nb) break;
-    float* row = S + (static_cast<size_t>(bh) * nb + i) * nb;
+  for (int a = 0; a < TM; ++a) {
+    const int i = i0 + (a < 4 ? ty * 4 + a : 64 + ty * 4 + a - 4);
+    if (i >= nb) continue;
+    float* row = S + (static_cast<size_t>(bh) * nb + i) * ld;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int j = j0 + tx * 4 + c;
-      if (j < nb) row[j] = acc[a][c] * scale;
+    for (int h = 0; h < 2; ++h) {
+      const int j = j0 + h * 64 + tx * 4;      // a multiple of 4; ld is too
+      if (j < ld)
+        *reinterpret_cast<float4*>(row + j) =
+            make_float4(acc[a][4 * h] * scale, acc[a][4 * h + 1] * scale, acc[a][4 * h + 2] * scale,
+                        acc[a][4 * h + 3] * scale);
     }
   }
 }
 
-// One warp per row of S: stage the row in shared memory, then select.
+// One warp per row of the score (or importance) matrix, read with row stride ld.
+template <int VPL>
 __global__ void __launch_bounds__(kRouteThreads)
-    select_rows_kernel(const float* __restrict__ S, int rows, int nb, float p, int k_min,
+    select_rows_kernel(const float* __restrict__ S, int ld, int rows, int nb, float p, int k_min,
                        int* __restrict__ kv_idx, int* __restrict__ kv_cnt,
                        unsigned long long* __restrict__ head_work, int* status, bool softmax) {
-  extern __shared__ float4 smem_f4[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* srow = reinterpret_cast<float*>(smem_f4) + static_cast<size_t>(warp) * nb;
   const int r = blockIdx.x * (kRouteThreads / 32) + warp;
   if (r >= rows) return;
-  const float* src = S + static_cast<size_t>(r) * nb;
-  for (int j = lane; j < nb; j += 32) srow[j] = src[j];
-  __syncwarp();
   const int bh = r / nb;
-  select_row(srow, nb, p, k_min, kv_idx + static_cast<size_t>(r) * nb, kv_cnt + r, head_work + bh,
-             status, lane, softmax);
+  select_row_reg<VPL>(S + static_cast<size_t>(r) * ld, nb, p, k_min, kv_idx + static_cast<size_t>(r) * nb,
+                      kv_cnt + r, head_work + bh, status, lane, softmax);
+}
+
+static cudaError_t launch_select(const float* S, int ld, int BH, int nb, float p, int k_min, int* kv_idx,
+                                 int* kv_cnt, unsigned long long* head_work, int* status, bool softmax,
+                                 cudaStream_t st) {
+  const int rows = BH * nb;
+  const int warps = kRouteThreads / 32;
+  const dim3 grid((rows + warps - 1) / warps);
+  const int vpl = (nb + 31) / 32;
+#define FVATTN_SELECT(V)                                                                         \
+  select_rows_kernel<V><<<grid, kRouteThreads, 0, st>>>(S, ld, rows, nb, p, k_min, kv_idx, kv_cnt, \
+                                                        head_work, status, softmax)
+  if (vpl <= 4) FVATTN_SELECT(4);
+  else if (vpl <= 8) FVATTN_SELECT(8);
+  else if (vpl <= 12) FVATTN_SELECT(12);
+  else if (vpl <= 16) FVATTN_SELECT(16);
+  else if (vpl <= 20) FVATTN_SELECT(20);
+  else if (vpl <= 24) FVATTN_SELECT(24);
+  else if (vpl <= 32) FVATTN_SELECT(32);
+  else if (vpl <= 40) FVATTN_SELECT(40);
+  else if (vpl <= 48) FVATTN_SELECT(48);
+  else if (vpl <= 64) FVATTN_SELECT(64);
+  else FVATTN_SELECT(128);
+#undef FVATTN_SELECT
+  return cudaGetLastError();
 }
 
 size_t route_scores_bytes(int BH, int nb) {
-  return static_cast<size_t>(BH) * nb * nb * sizeof(float);
+  return static_cast<size_t>(BH) * nb * scores_ld(nb) * sizeof(float);
 }
 
 cudaError_t launch_route_select(const float* qbar, const float* kbar, float* S, int BH, int nb, int d,
                                 float scale, float p, int k_min, int* kv_idx, int* kv_cnt,
                                 unsigned long long* head_work, int* status, cudaStream_t st) {
-  const size_t smem1 = static_cast<size_t>(2) * d * kTilePad * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(block_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem1));
+  const dim3 g1((nb + kTileN - 1) / kTileN, (nb + 16 * kScoreTM - 1) / (16 * kScoreTM), BH);
+  block_scores_kernel<kScoreTM><<<g1, kRouteThreads, 0, st>>>(qbar, kbar, nb, d, scale, S);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const dim3 g1((nb + kTile - 1) / kTile, (nb + kTile - 1) / kTile, BH);
-  block_scores_kernel<<<g1, kRouteThreads, smem1, st>>>(qbar, kbar, nb, d, scale, S);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const size_t smem2 = static_cast<size_t>(kRouteThreads / 32) * nb * sizeof(float);
-  e = cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem2));
-  if (e != cudaSuccess) return e;
-  const int rows = BH * nb;
-  const int warps = kRouteThreads / 32;
-  select_rows_kernel<<<(rows + warps - 1) / warps, kRouteThreads, smem2, st>>>(
-      S, rows, nb, p, k_min, kv_idx, kv_cnt, head_work, status, true);
-  return cudaGetLastError();
+  return launch_select(S, scores_ld(nb), BH, nb, p, k_min, kv_idx, kv_cnt, head_work, status, true, st);
 }
 
 // Top-p with the Top-k floor on given importance rows [BH, nb, nb] (no softmax).
 cudaError_t launch_select_topp(const float* rows_in, int BH, int nb, float p, int k_min, int* kv_idx,
                                int* kv_cnt, unsigned long long* head_work, int* status,
                                cudaStream_t st) {
-  const size_t smem = static_cast<size_t>(kRouteThreads / 32) * nb * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  const int rows = BH * nb;
-  const int warps = kRouteThreads / 32;
-  select_rows_kernel<<<(rows + warps - 1) / warps, kRouteThreads, smem, st>>>(
-      rows_in, rows, nb, p, k_min, kv_idx, kv_cnt, head_work, status, false);
-  return cudaGetLastError();
+  return launch_select(rows_in, nb, BH, nb, p, k_min, kv_idx, kv_cnt, head_work, status, false, st);
 }
 
 }  // namespace fvattn

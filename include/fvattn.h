@@ -31,6 +31,8 @@
  *   fvattn_hilbert_table  the permutation table of a grid   [FVAttn §3.1; GSRS §A.6]
  * Low-precision V [FVAttn §3.4]:
  *   fvattn_quantize_v       per-channel E4M3 codes and scales of the permuted V
+ *   fvattn_permute_quantize_v  the same codes straight from the raster-order V,
+ *                           fused with the block-order permutation
  *   fvattn_sparse_fwd_fp8v, fvattn_dense_fwd_fp8v
  *                           attention with that V (8-bit P.V on the tensor cores)
  *
@@ -239,6 +241,21 @@ FVATTN_API fvattn_status fvattn_dense_fwd(const void* qp, const void* kp, const 
 FVATTN_API fvattn_status fvattn_quantize_v(const void* vp, int B, int H, int N, int d, int block,
                                            uint8_t* vq, float* vscale, void* workspace,
                                            size_t workspace_bytes, void* stream);
+
+/* The block-order permutation of V fused with its per-channel FP8 quantization
+ * [FVAttn §3.1 block order; §3.4 the GPU quantizes V before attention]:
+ * v [B,H,N,128] bf16 in raster order (the input of fvattn_permute) in, vq
+ * [B,H,Npad,128] uint8 and vscale [B,H,128] fp32 out, equal bit for bit to
+ * fvattn_permute followed by fvattn_quantize_v (same definition of codes,
+ * scales, zero channels and zero pad rows; the grid's order, tiles or table,
+ * places the rows). V is read twice (channel maxima, then gather and encode)
+ * and the permuted bf16 V is never written: 1.5 B of traffic per V element
+ * less than the two calls. d must be 128 (FVATTN_ERR_UNSUPPORTED otherwise);
+ * v, vq and vscale 16-byte aligned and not overlapping; grid as for
+ * fvattn_permute. Workspace: fvattn_workspace_bytes(FVATTN_OP_QUANT_V, ...). */
+FVATTN_API fvattn_status fvattn_permute_quantize_v(const void* v, int B, int H, int N, int d,
+                                                   const fvattn_grid* grid, uint8_t* vq, float* vscale,
+                                                   void* workspace, size_t workspace_bytes, void* stream);
 
 /* Block-sparse attention forward with the FP8 V of fvattn_quantize_v:
  * fvattn_sparse_fwd's definition with V replaced by E4M3(vq) * vscale. qp, kp

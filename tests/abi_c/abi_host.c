@@ -55,6 +55,17 @@ int main(void) {
                           (void*)0x400000, NULL, NULL, B, H, N, d, FVATTN_BF16, block, 0.088f,
                           NULL, 0, NULL);
     CHECK(st == FVATTN_ERR_WORKSPACE, 34);
+    /* the fused V permutation + quantization: d = 128 only, and null outputs */
+    st = fvattn_permute_quantize_v((const void*)0x100000, B, H, N, 64, &g, (uint8_t*)0x10000000,
+                                   (float*)0x20000000, (void*)0x30000000, (size_t)1 << 20, NULL);
+    CHECK(st == FVATTN_ERR_UNSUPPORTED, 35);
+    st = fvattn_permute_quantize_v((const void*)0x100000, B, H, N, d, &g, NULL, NULL, NULL, 0, NULL);
+    CHECK(st == FVATTN_ERR_INVALID_ARG, 36);
+    /* the bounded-wait self-test needs its result buffer and a workspace */
+    st = fvattn_wait_selftest(NULL, (void*)0x30000000, 256, NULL);
+    CHECK(st == FVATTN_ERR_INVALID_ARG, 37);
+    st = fvattn_wait_selftest((int64_t*)0x100000, NULL, 0, NULL);
+    CHECK(st == FVATTN_ERR_WORKSPACE, 38);
   }
   {
     int s;

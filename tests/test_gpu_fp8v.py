@@ -99,6 +99,31 @@ def test_quantize_v_matches_oracle(w):
           f"{int((np.abs(Lp.e4m3_decode(got)) == 448).sum())} at +-448")
 
 
+@pytest.mark.parametrize("w", [ODD128, BS64, SINGLE, S.WORKLOADS["wan1.3b-480p"]], ids=lambda w: w.name)
+@pytest.mark.parametrize("order", ["tiles", "hilbert"])
+def test_permute_quantize_v_equals_permute_then_quantize(w, order):
+    """The fused call gives the codes and scales of fvattn_permute + fvattn_quantize_v,
+    bit for bit (including +-0 and the pad rows), and those of the oracle."""
+    q, k, v = S.make_qkv(w, device="cuda")
+    table = F.fvattn_hilbert_table(w.grid, w.block) if order == "hilbert" else None
+    grid = F.Grid.make(w.grid, w.tile, w.block, table=table)
+    npad = grid.nb * w.block
+    vp = torch.empty((w.B, w.H, npad, w.d), dtype=v.dtype, device="cuda")
+    F.fvattn_permute(v, vp, grid)
+    vq2, vs2 = _quant_gpu(w, vp)
+    vq = torch.full((w.B, w.H, npad, w.d), 0xA5, dtype=torch.uint8, device="cuda")
+    vs = torch.full((w.B, w.H, w.d), float("nan"), dtype=torch.float32, device="cuda")
+    ws = F.alloc_workspace(F.fvattn_workspace_bytes(F.FVATTN_OP_QUANT_V, w.B, w.H, w.N, w.d, w.block), "cuda")
+    for _ in range(2):      # the workspace's maxima are cleared by every call
+        F.fvattn_permute_quantize_v(v, grid, vq, vs, ws)
+        assert F.fvattn_workspace_status(ws) == F.FVATTN_OK
+        assert torch.equal(vq, vq2) and torch.equal(vs, vs2)
+    perm = table.cpu().numpy().astype(np.int64) if table is not None else _perm(w)
+    codes, scale = Lp.quantize_v(O.permute(_np(v), perm, w.block), w.N)
+    assert _same_codes(vq.cpu().numpy(), codes).all()
+    assert np.array_equal(vs.cpu().numpy(), scale)
+
+
 def test_quantize_v_sampled_720p_heads():
     # the 14B-720p V, full call; the oracle checks two heads completely
     w = S.WORKLOADS["wan14b-720p"]
