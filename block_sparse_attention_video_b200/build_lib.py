@@ -28,7 +28,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfvattn.so")
 HEADER = os.path.join(ROOT, "include", "fvattn.h")
 SOURCES = ["api.cu", "permute.cu", "route.cu", "attn_simt.cu", "attn_sm100.cu", "importance.cu",
-           "lvsa.cu", "hilbert.cu", "noalloc.cu", "quant.cu", "selftest.cu"]
+           "lvsa.cu", "hilbert.cu", "noalloc.cu", "quant.cu", "selftest.cu", "scores_tc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "-Xptxas", "-warn-spills", f"-I{os.path.join(ROOT, 'include')}"]

@@ -30,7 +30,7 @@ cudaError_t launch_attn_sm100(const CUtensorMap& tq, const CUtensorMap& tk, cons
                               const int* kv_idx, const int* kv_cnt,
                               uint32_t* ulist, int* ucnt, int* local_order,
                               unsigned long long* head_total, int* head_order, int BH, int N,
-                              int nb, int bs, float scale, int* status,
+                              int nb, int bs, int d, float scale, int* status,
                               unsigned long long* counter, int num_sms, cudaStream_t st);
 cudaError_t launch_block_importance(const float* blse, const float* lse, const int* kv_idx,
                                     const int* kv_cnt, int BH, int N, int bs, float* importance,
@@ -147,12 +147,13 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// [rows, 128] bf16, row stride 256 B; box = box_rows rows x 64 columns, 128-byte swizzle.
-bool make_row_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows) {
+// [rows, d] bf16 (d = 64 or 128), row stride 2d bytes; box = box_rows rows x 64
+// columns, 128-byte swizzle.
+bool make_row_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows, int d) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
-  cuuint64_t dims[2] = {128, rows};
-  cuuint64_t strides[1] = {256};
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), rows};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
@@ -224,8 +225,8 @@ fvattn_status attention_fwd(const void* qp, const void* kp, const void* vp, cons
     return FVATTN_ERR_INVALID_ARG;
   if (!valid_dtype(dtype) || !valid_sizes(B, H, N, d, block)) return FVATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return FVATTN_ERR_INVALID_ARG;
-  const bool tensor_core = dtype == FVATTN_BF16 && d == 128;
-  if (vscale && !tensor_core) return FVATTN_ERR_UNSUPPORTED;
+  const bool tensor_core = dtype == FVATTN_BF16;   // d is 64 or 128 (checked above)
+  if (vscale && !(tensor_core && d == 128)) return FVATTN_ERR_UNSUPPORTED;
   const size_t need = fvattn_workspace_bytes(sparse ? FVATTN_OP_SPARSE_FWD : FVATTN_OP_DENSE_FWD,
                                              B, H, N, d, block);
   const fvattn_status wst = check_ws(ws, ws_bytes, need);
@@ -245,8 +246,8 @@ fvattn_status attention_fwd(const void* qp, const void* kp, const void* vp, cons
   }
   const uint64_t rows = static_cast<uint64_t>(BH) * nb * block;
   CUtensorMap tq, tk, tv;
-  if (!make_row_map(&tq, qp, rows, 128) || !make_row_map(&tk, kp, rows, block) ||
-      !(vscale ? make_byte_row_map(&tv, vp, rows, block) : make_row_map(&tv, vp, rows, block)))
+  if (!make_row_map(&tq, qp, rows, 128, d) || !make_row_map(&tk, kp, rows, block, d) ||
+      !(vscale ? make_byte_row_map(&tv, vp, rows, block) : make_row_map(&tv, vp, rows, block, d)))
     return FVATTN_ERR_CUDA;
   const int sms = device_sm_count();
   if (sms <= 0) return FVATTN_ERR_CUDA;
@@ -265,7 +266,7 @@ fvattn_status attention_fwd(const void* qp, const void* kp, const void* vp, cons
   }
   return from_cuda(fvattn::launch_attn_sm100(
       tq, tk, tv, op, lse, block_lse, vscale, sparse ? kv_idx : nullptr, sparse ? kv_cnt : nullptr, ulist, ucnt,
-      local_order, head_total, head_order, BH, N, nb, block, scale, &hdr->status, &hdr->counter,
+      local_order, head_total, head_order, BH, N, nb, block, d, scale, &hdr->status, &hdr->counter,
       sms, st));
 }
 

@@ -68,10 +68,8 @@
 namespace fvattn {
 namespace sm100 {
 
-constexpr int HD = 128;
 constexpr int kUnitRows = 256;
-constexpr int kQTileBytes = 128 * HD * 2;   // 32 KB
-constexpr int kQHalfBytes = 128 * 128;      // 16 KB: 128 rows x 128 bytes
+constexpr int kQHalfBytes = 128 * 128;      // 16 KB: 128 rows x 64 columns (128 bytes)
 constexpr int kRingBytes = 128 * 1024;
 constexpr int kThreads = 384;
 constexpr int kRegsSoftmax = 184;
@@ -81,11 +79,14 @@ constexpr float kLn2 = 0.6931471805599453f;
 // A step covers 128 keys: one 128-token block, or two consecutive union entries
 // of 64-token blocks whose K (V) tiles are loaded into the two 64-row halves of
 // one 128-row stage. Every step is then an N = 128 S MMA and a K = 128 P.V.
-template <int BN, bool F8 = false>
+// HD = head dimension, 64 or 128: one or two 64-column (128-byte) halves per row.
+template <int BN, bool F8 = false, int HD = 128>
 struct Tile {
+  static constexpr int kHalves = HD / 64;
+  static constexpr int kQTileBytes = 128 * HD * 2;         // 32 KB (d 128), 16 KB (d 64)
   static constexpr int kStepKeys = 128;
   static constexpr int kBPS = kStepKeys / BN;              // union entries per step
-  static constexpr int kKVBytes = kStepKeys * HD * 2;      // 32 KB stage
+  static constexpr int kKVBytes = kStepKeys * HD * 2;      // 32 KB (16 KB) stage
   static constexpr int kKVHalf = kStepKeys * 128;          // one 64-column half of a stage
   static constexpr int kSubBytes = BN * 128;               // one entry's rows within a half
   static constexpr int kStages = kRingBytes / kKVBytes;
@@ -119,14 +120,14 @@ struct Params {
   unsigned long long* counter;
 };
 
-template <int BN>
+template <int BN, int HD>
 struct __align__(1024) Smem {
-  uint8_t q[2][kQTileBytes];
+  uint8_t q[2][Tile<BN, false, HD>::kQTileBytes];
   uint8_t kv[kRingBytes];
   uint64_t q_full[2];
   uint64_t q_empty[2];
-  uint64_t kv_full[Tile<BN>::kStages];
-  uint64_t kv_empty[Tile<BN>::kStages];
+  uint64_t kv_full[Tile<BN, false, HD>::kStages];
+  uint64_t kv_empty[Tile<BN, false, HD>::kStages];
   uint64_t s_full[2];
   uint64_t p_full[2][2];   // [slot][half of P]
   uint64_t o_full[2];
@@ -184,15 +185,17 @@ __device__ __forceinline__ uint32_t entry_at(const Unit& x, int k, const Params&
   return e;
 }
 
-template <int BN, bool F8>
+template <int BN, bool F8, int HD>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const Params P) {
-  using T = Tile<BN, F8>;
+  using T = Tile<BN, F8, HD>;
+  static_assert(HD == 64 || HD == 128, "head dimension 64 or 128");
+  static_assert(!F8 || HD == 128, "the E4M3-V path has d = 128");
   constexpr int kStages = T::kStages;
   extern __shared__ uint8_t smem_raw[];
-  Smem<BN>& sm = *reinterpret_cast<Smem<BN>*>(
+  Smem<BN, HD>& sm = *reinterpret_cast<Smem<BN, HD>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -274,9 +277,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int X = 0; X < 2; ++X) {
           if (!(X == 0 ? x.slot[0] : x.slot[1])) continue;
           if (!mbar_wait(&sm.q_empty[X], (qn[X] & 1) ^ 1, abort_flag, P.status)) { ok = false; break; }
-          mbar_arrive_expect_tx(&sm.q_full[X], kQTileBytes);
-          tma_load_2d(sm.q[X], &tm_q, &sm.q_full[X], 0, row0 + X * 128);
-          tma_load_2d(sm.q[X] + kQHalfBytes, &tm_q, &sm.q_full[X], 64, row0 + X * 128);
+          mbar_arrive_expect_tx(&sm.q_full[X], T::kQTileBytes);
+#pragma unroll
+          for (int hq = 0; hq < T::kHalves; ++hq)
+            tma_load_2d(sm.q[X] + hq * kQHalfBytes, &tm_q, &sm.q_full[X], 64 * hq, row0 + X * 128);
           ++qn[X];
         }
         const int ns = (x.cnt + T::kBPS - 1) / T::kBPS;
@@ -305,8 +309,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               const CUtensorMap* tm = t == 0 ? &tm_k : &tm_v;
 #pragma unroll
               for (int h = 0; h < T::kBPS; ++h) {
-                tma_load_2d(dst + h * T::kSubBytes, tm, &sm.kv_full[s], 0, kvrow[h]);
-                tma_load_2d(dst + T::kKVHalf + h * T::kSubBytes, tm, &sm.kv_full[s], 64, kvrow[h]);
+#pragma unroll
+                for (int hq = 0; hq < T::kHalves; ++hq)
+                  tma_load_2d(dst + hq * T::kKVHalf + h * T::kSubBytes, tm, &sm.kv_full[s], 64 * hq, kvrow[h]);
               }
             }
             ++it;
@@ -547,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float f = need ? ex2_approx(m_run - m_new) : 1.f;
               l_run *= f;
 #pragma unroll 1
-              for (int c = 0; c < 4; ++c) {
+              for (int c = 0; c < HD / 32; ++c) {
                 uint32_t o[32];
                 tmem_ld32(tO + c * 32, o);
                 tmem_wait_ld();
@@ -646,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const size_t grow = static_cast<size_t>(x.bh) * P.npad + qrow;
       uint4* orow = reinterpret_cast<uint4*>(P.out + grow * HD);
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < HD / 32; ++c) {
         uint32_t o[32];
         tmem_ld32(tO + c * 32, o);
         tmem_wait_ld();
@@ -819,16 +824,16 @@ __global__ void __launch_bounds__(1024)
 }
 
 // ---------------------------------------------------------------- launcher
-template <int BN, bool F8>
+template <int BN, bool F8, int HD>
 static cudaError_t launch_bn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const sm100::Params& P, int num_sms, cudaStream_t st) {
-  const size_t smem = sizeof(sm100::Smem<BN>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(sm100::attn_fwd_sm100_kernel<BN, F8>,
+  const size_t smem = sizeof(sm100::Smem<BN, HD>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(sm100::attn_fwd_sm100_kernel<BN, F8, HD>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int grid = max(1, min(num_sms, P.total_units));
-  sm100::attn_fwd_sm100_kernel<BN, F8><<<grid, sm100::kThreads, smem, st>>>(tq, tk, tv, P);
+  sm100::attn_fwd_sm100_kernel<BN, F8, HD><<<grid, sm100::kThreads, smem, st>>>(tq, tk, tv, P);
   return cudaGetLastError();
 }
 
@@ -837,7 +842,7 @@ cudaError_t launch_attn_sm100(const CUtensorMap& tq, const CUtensorMap& tk, cons
                               const int* kv_idx, const int* kv_cnt,
                               uint32_t* ulist, int* ucnt, int* local_order,
                               unsigned long long* head_total, int* head_order, int BH, int N,
-                              int nb, int bs, float scale, int* status,
+                              int nb, int bs, int d, float scale, int* status,
                               unsigned long long* counter, int num_sms, cudaStream_t st) {
   const int G = sm100::kUnitRows / bs;
   const int ngroups = (nb + G - 1) / G;
@@ -870,10 +875,13 @@ cudaError_t launch_attn_sm100(const CUtensorMap& tq, const CUtensorMap& tk, cons
   P.status = status;
   P.counter = counter;
   if (vscale)
-    return bs == 64 ? launch_bn<64, true>(tq, tk, tv, P, num_sms, st)
-                    : launch_bn<128, true>(tq, tk, tv, P, num_sms, st);
-  return bs == 64 ? launch_bn<64, false>(tq, tk, tv, P, num_sms, st)
-                  : launch_bn<128, false>(tq, tk, tv, P, num_sms, st);
+    return bs == 64 ? launch_bn<64, true, 128>(tq, tk, tv, P, num_sms, st)
+                    : launch_bn<128, true, 128>(tq, tk, tv, P, num_sms, st);
+  if (d == 64)
+    return bs == 64 ? launch_bn<64, false, 64>(tq, tk, tv, P, num_sms, st)
+                    : launch_bn<128, false, 64>(tq, tk, tv, P, num_sms, st);
+  return bs == 64 ? launch_bn<64, false, 128>(tq, tk, tv, P, num_sms, st)
+                  : launch_bn<128, false, 128>(tq, tk, tv, P, num_sms, st);
 }
 
 }  // namespace fvattn

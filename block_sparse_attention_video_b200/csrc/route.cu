@@ -1,15 +1,15 @@
 // route.cu -- block scores, softmax and Top-p / Top-k-floor selection
 // [FVAttn §2.1, §2.2 Eq. (1), §3.1; GSRS §5.2, §5.3, §A.4].
 //
-// Two kernels, each at high occupancy:
-//   1. block_scores_kernel: S[b,h,i,j] = scale * qbar_i . kbar_j for every pair
-//      of blocks, fp32, as a 128 x 128 tiled SIMT product (8 x 8 outputs per
-//      thread from register-held operands, d staged 32 at a time k-major in
-//      shared memory); S goes to the route workspace with its row stride padded
-//      to a multiple of 4 so that every thread stores whole float4s.
+// Two kernels:
+//   1. block_scores_tc_kernel (scores_tc.cu): S[b,h,i,j] = scale * qbar_i . kbar_j
+//      for every pair of blocks on the tensor cores, with fp32-level accuracy
+//      from a split of each operand into two TF32 parts; S goes to the route
+//      workspace with its row stride padded to a multiple of 4 floats.
 //   2. select_rows_kernel: one warp per (b, h, query block) row, the row held in
 //      registers (32 per lane and up to 48 values per lane; longer rows are staged
-//      in shared memory): max-subtracted softmax (expf, fixed-order warp sums),
+//      in shared memory): max-subtracted softmax (the scores arrive as base-2
+//      logits, so exp2f; fixed-order warp sums),
 //      then the Top-p cut found without sorting: the largest value v* with
 //      F(v*) = sum_{s_j >= v*} s_j >= p. F is evaluated with each lane's fp32
 //      partial sum (fixed order) rounded to a 2^-31 fixed point and added
@@ -91,7 +91,7 @@ __device__ void select_row_reg(const float* __restrict__ src, int nb, float p, i
     float z = 0.f;
 #pragma unroll
     for (int t = 0; t < VPL; ++t) {
-      v[t] = expf(v[t] - m);
+      v[t] = exp2f(v[t] - m);   // the row holds base-2 logits: 2^(x log2 e) = e^x
       z += v[t];
     }
     z = warp_sum(z);
@@ -158,6 +158,7 @@ __device__ void select_row_reg(const float* __restrict__ src, int nb, float p, i
   int cnt;
   float thr;      // selected: v > thr, plus the first take_eq entries equal to thr
   int take_eq;
+  bool tie_split = false;   // some, not all, of the entries equal to thr are taken
   if (p >= 1.f || k_min >= nb) {
     cnt = nb;
     thr = -1.f;
@@ -166,6 +167,7 @@ __device__ void select_row_reg(const float* __restrict__ src, int nb, float p, i
     int n_p;
     float vstar = 0.f;
     int cgt = 0;
+    int ceq_star = 1;
     const uint32_t target = to_fix(p);
     uint32_t total;
     int call;
@@ -192,6 +194,7 @@ __device__ void select_row_reg(const float* __restrict__ src, int nb, float p, i
       vstar = __uint_as_float(lo);
       cgt = c_hi;
       const int ceq = c_lo - c_hi;
+      ceq_star = ceq;
       const uint32_t fstar = to_fix(vstar);
       int need = 1;
       uint32_t acc = f_hi + fstar;
@@ -205,6 +208,7 @@ __device__ void select_row_reg(const float* __restrict__ src, int nb, float p, i
     } else if (cnt == n_p) {
       thr = vstar;
       take_eq = cnt - cgt;
+      tie_split = take_eq < ceq_star;
     } else {
       uint32_t lo = vmin, hi = vmax + 1u;          // count(lo) >= cnt > count(hi)
       int c_lo = nb, c_hi = 0;
@@ -217,24 +221,45 @@ __device__ void select_row_reg(const float* __restrict__ src, int nb, float p, i
       if (c_lo - c_hi == 1) lo = only_below(hi);
       thr = __uint_as_float(lo);
       take_eq = cnt - c_hi;
+      tie_split = take_eq < c_lo - c_hi;
     }
   }
 
-  // compaction in ascending block index
+  // compaction in ascending block index (cnt and tie_split are warp-uniform)
   const unsigned lt_mask = (1u << lane) - 1u;
-  int written = 0, eq_seen = 0;
+  int written = 0;
+  if (cnt == nb) {
+    // every block: the list is 0 .. nb-1
 #pragma unroll
-  for (int t = 0; t < VPL; ++t) {
-    const int j = t * 32 + lane;
-    const bool valid = j < nb;
-    const bool eq = valid && v[t] == thr;
-    const unsigned eqb = __ballot_sync(0xffffffffu, eq);
-    const int eq_rank = eq_seen + __popc(eqb & lt_mask);
-    const bool sel = valid && (v[t] > thr || (eq && eq_rank < take_eq));
-    const unsigned sb = __ballot_sync(0xffffffffu, sel);
-    if (sel) out_idx[written + __popc(sb & lt_mask)] = j;
-    written += __popc(sb);
-    eq_seen += __popc(eqb);
+    for (int t = 0; t < VPL; ++t) {
+      const int j = t * 32 + lane;
+      if (j < nb) out_idx[j] = j;
+    }
+    written = nb;
+  } else if (!tie_split) {
+    // every entry equal to thr is taken: the selection is v >= thr (pads, -1, are below)
+#pragma unroll
+    for (int t = 0; t < VPL; ++t) {
+      const bool sel = v[t] >= thr;
+      const unsigned sb = __ballot_sync(0xffffffffu, sel);
+      if (sel) out_idx[written + __popc(sb & lt_mask)] = t * 32 + lane;
+      written += __popc(sb);
+    }
+  } else {
+    int eq_seen = 0;
+#pragma unroll
+    for (int t = 0; t < VPL; ++t) {
+      const int j = t * 32 + lane;
+      const bool valid = j < nb;
+      const bool eq = valid && v[t] == thr;
+      const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+      const int eq_rank = eq_seen + __popc(eqb & lt_mask);
+      const bool sel = valid && (v[t] > thr || (eq && eq_rank < take_eq));
+      const unsigned sb = __ballot_sync(0xffffffffu, sel);
+      if (sel) out_idx[written + __popc(sb & lt_mask)] = j;
+      written += __popc(sb);
+      eq_seen += __popc(eqb);
+    }
   }
   if (lane == 0) {
     *out_cnt = cnt;
@@ -243,95 +268,11 @@ __device__ void select_row_reg(const float* __restrict__ src, int nb, float p, i
   }
 }
 
-constexpr int kTileN = 128;      // score tile: 16*TM query blocks x 128 key blocks
-constexpr int kKc = 32;          // d staged 32 at a time
-constexpr int kTilePad = kTileN + 4;
-#ifndef FVATTN_SCORE_TM
-#define FVATTN_SCORE_TM 8
-#endif
-constexpr int kScoreTM = FVATTN_SCORE_TM;   // query blocks per thread (4 or 8)
-
 // Row stride of the block score matrix: nb padded to a multiple of 4 floats.
 __host__ __device__ __forceinline__ int scores_ld(int nb) { return (nb + 3) & ~3; }
 
-// S tile = scale * Qtile . Ktile^T over d; 16 x 16 threads, each TM x 8 outputs:
-// rows ty*4 + {0..3} (and 64 + ty*4 + {0..3} when TM = 8), columns tx*4 + {0..3}
-// and 64 + tx*4 + {0..3}, so that a warp's shared-memory reads of a k-slice are
-// contiguous 256-byte runs. Means past nb are read as zero; their (finite)
-// scores land in rows past nb, which are not stored, or in columns past nb,
-// which the selection never reads.
-template <int TM>
-__global__ void __launch_bounds__(kRouteThreads, TM == 8 ? 2 : 3)
-    block_scores_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar, int nb, int d,
-                        float scale, float* __restrict__ S) {
-  constexpr int kTileM = 16 * TM;
-  __shared__ __align__(16) float qs[kKc][kTileM + 4];
-  __shared__ __align__(16) float ks[kKc][kTilePad];
-  const int bh = blockIdx.z;
-  const int i0 = blockIdx.y * kTileM, j0 = blockIdx.x * kTileN;
-  const float* qb = qbar + static_cast<size_t>(bh) * nb * d;
-  const float* kb = kbar + static_cast<size_t>(bh) * nb * d;
-  const int ld = scores_ld(nb);
-  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-  float acc[TM][8];
-#pragma unroll
-  for (int a = 0; a < TM; ++a)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[a][c] = 0.f;
-  for (int k0 = 0; k0 < d; k0 += kKc) {
-    // rows of the tile are the fastest index so that the transposing stores hit distinct banks
-    for (int e = threadIdx.x; e < kTileN * (kKc / 4); e += kRouteThreads) {
-      const int r = e % kTileN, cl = (e / kTileN) * 4, c = k0 + cl;
-      float4 ka = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j0 + r < nb) ka = *reinterpret_cast<const float4*>(kb + static_cast<size_t>(j0 + r) * d + c);
-      ks[cl + 0][r] = ka.x;
-      ks[cl + 1][r] = ka.y;
-      ks[cl + 2][r] = ka.z;
-      ks[cl + 3][r] = ka.w;
-      if (r < kTileM) {
-        float4 qa = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (i0 + r < nb) qa = *reinterpret_cast<const float4*>(qb + static_cast<size_t>(i0 + r) * d + c);
-        qs[cl + 0][r] = qa.x;
-        qs[cl + 1][r] = qa.y;
-        qs[cl + 2][r] = qa.z;
-        qs[cl + 3][r] = qa.w;
-      }
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int kk = 0; kk < kKc; ++kk) {
-      float qv[TM];
-      const float4 q0 = *reinterpret_cast<const float4*>(&qs[kk][ty * 4]);
-      qv[0] = q0.x; qv[1] = q0.y; qv[2] = q0.z; qv[3] = q0.w;
-      if constexpr (TM == 8) {
-        const float4 q1 = *reinterpret_cast<const float4*>(&qs[kk][64 + ty * 4]);
-        qv[4] = q1.x; qv[5] = q1.y; qv[6] = q1.z; qv[7] = q1.w;
-      }
-      const float4 k0v = *reinterpret_cast<const float4*>(&ks[kk][tx * 4]);
-      const float4 k1v = *reinterpret_cast<const float4*>(&ks[kk][64 + tx * 4]);
-      const float kf[8] = {k0v.x, k0v.y, k0v.z, k0v.w, k1v.x, k1v.y, k1v.z, k1v.w};
-#pragma unroll
-      for (int a = 0; a < TM; ++a)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[a][c] = fmaf(qv[a], kf[c], acc[a][c]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int a = 0; a < TM; ++a) {
-    const int i = i0 + (a < 4 ? ty * 4 + a : 64 + ty * 4 + a - 4);
-    if (i >= nb) continue;
-    float* row = S + (static_cast<size_t>(bh) * nb + i) * ld;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int j = j0 + h * 64 + tx * 4;      // a multiple of 4; ld is too
-      if (j < ld)
-        *reinterpret_cast<float4*>(row + j) =
-            make_float4(acc[a][4 * h] * scale, acc[a][4 * h + 1] * scale, acc[a][4 * h + 2] * scale,
-                        acc[a][4 * h + 3] * scale);
-    }
-  }
-}
+cudaError_t launch_block_scores_tc(const float* qbar, const float* kbar, int BH, int nb, int d, float scale,
+                                   int ld, float* S, int* status, cudaStream_t st);
 
 // One warp per row of the score (or importance) matrix, read with row stride ld.
 template <int VPL>
@@ -379,9 +320,9 @@ size_t route_scores_bytes(int BH, int nb) {
 cudaError_t launch_route_select(const float* qbar, const float* kbar, float* S, int BH, int nb, int d,
                                 float scale, float p, int k_min, int* kv_idx, int* kv_cnt,
                                 unsigned long long* head_work, int* status, cudaStream_t st) {
-  const dim3 g1((nb + kTileN - 1) / kTileN, (nb + 16 * kScoreTM - 1) / (16 * kScoreTM), BH);
-  block_scores_kernel<kScoreTM><<<g1, kRouteThreads, 0, st>>>(qbar, kbar, nb, d, scale, S);
-  cudaError_t e = cudaGetLastError();
+  // base-2 logits: the selection's softmax then takes exp2f
+  cudaError_t e = launch_block_scores_tc(qbar, kbar, BH, nb, d, scale * 1.4426950408889634f, scores_ld(nb), S,
+                                         status, st);
   if (e != cudaSuccess) return e;
   return launch_select(S, scores_ld(nb), BH, nb, p, k_min, kv_idx, kv_cnt, head_work, status, true, st);
 }

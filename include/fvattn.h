@@ -197,11 +197,11 @@ FVATTN_API fvattn_status fvattn_route_noalloc(const void* q, const void* k, int 
  * lse it gives the exact block importance (fvattn_block_importance). NULL to
  * skip; the tensor-core kernel then does no extra work. kv_idx/kv_cnt as produced by fvattn_route (any order
  * of entries within a row is accepted). scale > 0 (1/sqrt(d) is the usual).
- * BF16 with d == 128 (block 64 or 128) runs the tcgen05/TMEM tensor-core
+ * BF16 (d 64 or 128, block 64 or 128) runs the tcgen05/TMEM tensor-core
  * kernel (bf16 MMA, fp32 accumulation and softmax, P rounded to bf16); it
  * processes 256 query rows at a time over the union of their blocks' lists,
- * masking each row to its own block's list. d == 64 and FP32 run the SIMT
- * kernel (fp32 throughout).
+ * masking each row to its own block's list. FP32 runs the SIMT kernel (fp32
+ * throughout; the tensor cores have no fp32 path with that accuracy).
  * Workspace: fvattn_workspace_bytes(FVATTN_OP_SPARSE_FWD, ...). */
 FVATTN_API fvattn_status fvattn_sparse_fwd(const void* qp, const void* kp, const void* vp,
                                 void* op, float* lse, float* block_lse,

@@ -67,6 +67,10 @@ TINY_BF16 = S.Workload("tiny-bf16-d128", 1, 2, 128, "bf16", (4, 16, 16), (1, 8, 
 PEAKY = S.Workload("peaky-rescale", 1, 3, 128, "bf16", (4, 16, 24), (1, 8, 16), 128, 0.97, 2,
                    seed=15, gen="gauss", peaky_head=2, peaky_scale=8.0)
 BS64 = S.Workload("bs64-d128", 2, 2, 128, "bf16", (5, 12, 20), (1, 8, 8), 64, 0.8, 3, seed=16)
+# d = 64 on the tensor cores: 128-token blocks with a ragged tail, and large logits (O rescale)
+D64 = S.Workload("d64-bs128", 2, 3, 64, "bf16", (3, 10, 14), (2, 8, 8), 128, 0.85, 2, seed=17)
+PEAKY_D64 = S.Workload("peaky-d64", 1, 3, 64, "bf16", (4, 16, 24), (1, 8, 16), 128, 0.97, 2,
+                       seed=18, gen="gauss", peaky_head=2, peaky_scale=8.0)
 
 
 # ----------------------------------------------------------------- permutation
@@ -156,7 +160,7 @@ def _sample_blocks(w, nb, cnt=None, per_head=6, seed=0):
     return out
 
 
-@pytest.mark.parametrize("w", [S.WORKLOADS["tiny"], ODD, ODD128, SINGLE, TINY_BF16, PEAKY, BS64],
+@pytest.mark.parametrize("w", [S.WORKLOADS["tiny"], ODD, ODD128, SINGLE, TINY_BF16, PEAKY, BS64, D64, PEAKY_D64],
                          ids=lambda w: w.name)
 def test_sparse_and_dense_attention_all_blocks(w):
     q, k, v = S.make_qkv(w, device="cuda")
@@ -198,8 +202,8 @@ def test_tensor_core_attention_sampled(name):
                      BF16_MAX_ABS, BF16_MEAN_ABS)
 
 
-def test_sparse_with_full_lists_is_bitwise_dense():
-    w = ODD128
+@pytest.mark.parametrize("w", [ODD128, D64], ids=lambda w: w.name)
+def test_sparse_with_full_lists_is_bitwise_dense(w):
     q, k, v = S.make_qkv(w, device="cuda")
     grid = F.Grid.make(w.grid, w.tile, w.block)
     nb = grid.nb
