@@ -43,27 +43,41 @@ METRIC = "sparse attn ms/call & effective TFLOP/s (Wan-14B 720p shape) vs own de
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
-# launch from a one-pass ncu capture, per workload, with the sha256 prefix of
-# the kernel source they were taken on. They are reported only while the source
-# is unchanged; after any change the traffic is unknown and reported as null.
+# launch from a one-pass ncu capture on the Wan-14B 480p shape (the size a
+# capture may hold), with the algorithmic bytes of that launch (Q, K, V read
+# once, O written once) and the sha256 prefix of the kernel source it was taken
+# on. A 720p launch's traffic is reported as the 480p traffic scaled by the ratio
+# of algorithmic bytes: the working set of the work units in flight (about one
+# head's K and V) fits in L2 at both sizes, so the re-read factor carries over.
+# After any change of the source the traffic is unknown and reported as null.
 ATTN_TRAFFIC = {
-    "wan14b-720p": {"bytes": 2.55e9 + 764.74e6, "src": "7a980de0684eea7e"},
-    "wan14b-720p/fp8v": {"bytes": 2.02e9 + 758.44e6, "src": "7a980de0684eea7e"},
+    # 1,021,980,416 read + 320,834,816 written; Q, K, V, O at 2 B x 40 x 256 x 128 x 128
+    "bf16": {"bytes_480p": 1021980416 + 320834816, "algorithmic_480p": 4 * 40 * 256 * 128 * 128 * 2,
+             "src": "75a9d8b8ec84c740"},
+    # 847,159,296 read + 316,532,224 written; Q, K, O at 2 B and the E4M3 V at 1 B
+    "fp8v": {"bytes_480p": 847159296 + 316532224, "algorithmic_480p": 7 * 40 * 256 * 128 * 128,
+             "src": "75a9d8b8ec84c740"},
 }
 ATTN_SRC = os.path.join(ROOT, "block_sparse_attention_video_b200", "csrc", "attn_sm100.cu")
 
 
-def _attn_traffic(workload: str):
+def _attn_traffic(kind: str, algorithmic_bytes: float):
+    """(scaled DRAM bytes per launch, note) for the current kernel source, or (None, why)."""
     import hashlib
-    rec = ATTN_TRAFFIC.get(workload)
-    if rec is None:
-        return None
+    rec = ATTN_TRAFFIC.get(kind)
+    if rec is None or rec["bytes_480p"] is None:
+        return None, "no capture recorded"
     try:
         with open(ATTN_SRC, "rb") as f:
             sha = hashlib.sha256(f.read()).hexdigest()
     except OSError:
-        return None
-    return rec["bytes"] if sha.startswith(rec["src"]) else None
+        return None, "kernel source not found"
+    if not sha.startswith(rec["src"]):
+        return None, "kernel source changed since the capture"
+    ratio = rec["bytes_480p"] / rec["algorithmic_480p"]
+    return ratio * algorithmic_bytes, (f"ncu one-pass DRAM bytes at the Wan-14B 480p shape "
+                                       f"({rec['bytes_480p'] / 1e9:.3f} GB, {ratio:.3f}x its algorithmic bytes), "
+                                       f"scaled to this launch's algorithmic bytes")
 
 
 def _peaks():
@@ -355,11 +369,13 @@ def run_fp8v(F, w, path, stream, warmup, eff, q, k, v):
 def run_hilbert(F, w, q, k, v, stream, warmup, eff_flops_fn):
     """The same call with blocks in Hilbert-curve order instead of 3-D tiles."""
     dev = q.device
+    hpath = F.FVAttnPath(w.B, w.H, w.grid, w.tile, w.block, w.d, torch.bfloat16, w.p, w.k_min, device=dev,
+                         order="hilbert")
+    # the table build alone (once per grid), its buffers already cached by the first build
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    hpath = F.FVAttnPath(w.B, w.H, w.grid, w.tile, w.block, w.d, torch.bfloat16, w.p, w.k_min, device=dev,
-                         order="hilbert")
+    F.fvattn_hilbert_table(w.grid, w.block, dev)
     t1.record(stream)
     torch.cuda.synchronize()
     table_ms = t0.elapsed_time(t1)
@@ -605,6 +621,8 @@ def run_fvattn(args):
     pk = _peaks()
     achieved = eff / (ms_attn * 1e-3) / 1e12
     hb = hbm_bytes(w, path.nb, int(cnt_np.astype(np.int64).sum()))
+    attn_alg_bytes = 4 * w.B * w.H * path.nb * w.block * w.d * 2
+    traffic_bf16, traffic_bf16_note = _attn_traffic("bf16", attn_alg_bytes)
     hbm_ms = ms_route + ms_vperm + ms_inv
     hbm_achieved = (hb["route"] + hb["permute_v"] + hb["inverse"]) / (hbm_ms * 1e-3) / 1e9
     line = {
@@ -630,8 +648,9 @@ def run_fvattn(args):
                      "peak": pk["bf16_sus"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_sus"],
                      "peak_kind": f"{pk['source']} bf16 sustained (kernel timed inside a long step)",
                      "frac_of_burst_peak": achieved / pk["bf16"],
-                     "traffic": _attn_traffic(w.name), "traffic_unit": "bytes per launch (DRAM read + write)",
-                     "algorithmic_bytes": 4 * w.B * w.H * path.nb * w.block * w.d * 2},
+                     "traffic": traffic_bf16, "traffic_note": traffic_bf16_note,
+                     "traffic_unit": "bytes per launch (DRAM read + write)",
+                     "algorithmic_bytes": attn_alg_bytes},
         "roofline_hbm": {"bound": "hbm", "kernels": "route (gather + pool, block scores, select) + V permute + "
                                                     "inverse permute",
                          "achieved": hbm_achieved, "peak": pk["hbm"], "unit": "GB/s",
@@ -658,7 +677,7 @@ def run_fvattn(args):
         p8 = pk["bf16_sus"] * 4.0 / 3.0
         fp8v["roofline"] = {"bound": "tensor", "kernel": "attn_fwd_sm100_kernel (E4M3 P.V)", "achieved": a8,
                             "peak": p8, "unit": "TFLOP/s", "frac": a8 / p8,
-                            "traffic": _attn_traffic(w.name + "/fp8v"),
+                            "traffic": _attn_traffic("fp8v", 7 * w.B * w.H * path.nb * w.block * w.d)[0],
                             # Q, K read (2 B each), E4M3 V read (1 B), O written (2 B) per element
                             "algorithmic_bytes": 7 * w.B * w.H * path.nb * w.block * w.d,
                             "peak_kind": f"{pk['source']} bf16 sustained x 4/3 (half the FLOPs at the "

@@ -40,13 +40,14 @@ def test_sweep_covers_p_kmin_and_block_sizes():
 def test_traffic_is_reported_only_for_the_captured_source():
     with open(bench.ATTN_SRC, "rb") as f:
         sha = hashlib.sha256(f.read()).hexdigest()
-    for key, rec in bench.ATTN_TRAFFIC.items():
-        got = bench._attn_traffic(key)
-        if sha.startswith(rec["src"]):
-            assert got == rec["bytes"]
+    for kind, rec in bench.ATTN_TRAFFIC.items():
+        got, note = bench._attn_traffic(kind, 2.0e9)
+        if rec["bytes_480p"] is not None and sha.startswith(rec["src"]):
+            assert got == pytest.approx(rec["bytes_480p"] / rec["algorithmic_480p"] * 2.0e9)
+            assert "480p" in note
         else:
-            assert got is None
-    assert bench._attn_traffic("no-such-workload") is None
+            assert got is None and note
+    assert bench._attn_traffic("no-such-kind", 1.0) == (None, "no capture recorded")
 
 
 def test_reference_arm_line(capsys):

@@ -67,6 +67,9 @@ TINY_BF16 = S.Workload("tiny-bf16-d128", 1, 2, 128, "bf16", (4, 16, 16), (1, 8, 
 PEAKY = S.Workload("peaky-rescale", 1, 3, 128, "bf16", (4, 16, 24), (1, 8, 16), 128, 0.97, 2,
                    seed=15, gen="gauss", peaky_head=2, peaky_scale=8.0)
 BS64 = S.Workload("bs64-d128", 2, 2, 128, "bf16", (5, 12, 20), (1, 8, 8), 64, 0.8, 3, seed=16)
+# 64-token blocks with an odd block count (the last unit's second block is past the end) and
+# an odd number of units (3 heads x 9), so the last round of unit pairs has an idle slot
+BS64_ODD = S.Workload("bs64-odd-units", 1, 3, 128, "bf16", (4, 16, 17), (1, 8, 8), 64, 0.7, 2, seed=19)
 # d = 64 on the tensor cores: 128-token blocks with a ragged tail, and large logits (O rescale)
 D64 = S.Workload("d64-bs128", 2, 3, 64, "bf16", (3, 10, 14), (2, 8, 8), 128, 0.85, 2, seed=17)
 PEAKY_D64 = S.Workload("peaky-d64", 1, 3, 64, "bf16", (4, 16, 24), (1, 8, 16), 128, 0.97, 2,
@@ -160,7 +163,8 @@ def _sample_blocks(w, nb, cnt=None, per_head=6, seed=0):
     return out
 
 
-@pytest.mark.parametrize("w", [S.WORKLOADS["tiny"], ODD, ODD128, SINGLE, TINY_BF16, PEAKY, BS64, D64, PEAKY_D64],
+@pytest.mark.parametrize("w", [S.WORKLOADS["tiny"], ODD, ODD128, SINGLE, TINY_BF16, PEAKY, BS64, BS64_ODD, D64,
+                               PEAKY_D64],
                          ids=lambda w: w.name)
 def test_sparse_and_dense_attention_all_blocks(w):
     q, k, v = S.make_qkv(w, device="cuda")
