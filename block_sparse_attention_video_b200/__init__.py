@@ -62,7 +62,7 @@ EXPORTED = ("fvattn_workspace_bytes", "fvattn_permute", "fvattn_route", "fvattn_
             "fvattn_select_topp", "fvattn_lvsa_lists", "fvattn_hilbert_table", "fvattn_quantize_v",
             "fvattn_sparse_fwd_fp8v", "fvattn_dense_fwd_fp8v",
             "fvattn_workspace_status", "fvattn_status_string", "fvattn_wait_selftest",
-            "fvattn_permute_quantize_v")
+            "fvattn_permute_quantize_v", "fvattn_order_lists_by_importance")
 
 
 class Grid(ctypes.Structure):
@@ -103,6 +103,9 @@ _lib.fvattn_route_noalloc.argtypes = [_c_void_p, _c_void_p, _c_int, _c_int, _c_i
                                       ctypes.POINTER(Grid), _c_float, _c_int, _c_void_p, _c_void_p,
                                       _c_void_p, _c_void_p, _c_void_p, _c_void_p]
 _lib.fvattn_route_noalloc.restype = _c_int
+_lib.fvattn_order_lists_by_importance.argtypes = [_c_void_p, _c_void_p] + [_c_int] * 5 + [_c_void_p, _c_size_t,
+                                                                                       _c_void_p]
+_lib.fvattn_order_lists_by_importance.restype = _c_int
 _lib.fvattn_sparse_fwd.argtypes = [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                                    _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int,
                                    _c_int, _c_int, _c_float, _c_void_p, _c_size_t, _c_void_p]
@@ -275,6 +278,22 @@ def _check_route_buffers(q, k, grid, kv_idx, kv_cnt, head_work, qp_out, kp_out):
     _check_lists(kv_idx, kv_cnt, head_work, dev, B, H, nb)
     for t, name in ((qp_out, "qp_out"), (kp_out, "kp_out")):
         _expect(t, name, dev, (B, H, nb * grid.block, d), q.dtype, optional=True)
+
+
+def fvattn_order_lists_by_importance(kv_idx, kv_cnt, N: int, d: int, block: int, workspace, stream=None):
+    """Reorders the lists of the preceding fvattn_route call made with this workspace
+    by descending block score (ties by block index), in place."""
+    _need_cuda(kv_idx, kv_cnt, workspace)
+    dev = kv_cnt.device
+    B, H, nb = kv_cnt.shape
+    if nb != _nb(N, block):
+        raise ValueError(f"kv_cnt has {nb} blocks per row, expected {_nb(N, block)}")
+    _check_lists(kv_idx, kv_cnt, None, dev, B, H, nb)
+    _expect_ws(workspace, dev)
+    _check(_call(dev, _lib.fvattn_order_lists_by_importance, _ptr(kv_idx), _ptr(kv_cnt), B, H, N, d, block,
+                 _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream, dev)),
+           "fvattn_order_lists_by_importance")
+    return kv_idx
 
 
 def fvattn_route_noalloc(q, k, grid: Grid, p: float, k_min: int, kv_idx, kv_cnt, head_work,

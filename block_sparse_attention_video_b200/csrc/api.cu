@@ -46,6 +46,8 @@ cudaError_t launch_quantize_v(const void* v, int BH, int N, int npad, uint8_t* v
                               unsigned int* amax_bits, cudaStream_t st);
 size_t vquant_ws_bytes(int BH);
 cudaError_t launch_wait_selftest(long long* out, int* status, cudaStream_t st);
+cudaError_t launch_order_lists(const float* S, int BH, int nb, int* kv_idx, const int* kv_cnt, int* status,
+                               cudaStream_t st);
 cudaError_t launch_permute_quantize_v(const void* v, int BH, int N, int bs, const TileGeom& g, uint8_t* vq,
                                       float* vscale, unsigned int* amax_bits, cudaStream_t st);
 int hilbert_bits(int extent);
@@ -344,6 +346,21 @@ fvattn_status fvattn_route(const void* q, const void* k, int B, int H, int N, in
                                   reinterpret_cast<unsigned long long*>(head_work), &hdr->status,
                                   st);
   return from_cuda(e);
+}
+
+fvattn_status fvattn_order_lists_by_importance(int32_t* kv_idx, const int32_t* kv_cnt, int B, int H, int N,
+                                               int d, int block, void* route_workspace,
+                                               size_t workspace_bytes, void* stream) {
+  if (!kv_idx || !kv_cnt || !aligned(kv_idx, 4) || !aligned(kv_cnt, 4)) return FVATTN_ERR_INVALID_ARG;
+  if (!valid_sizes(B, H, N, d, block)) return FVATTN_ERR_INVALID_ARG;
+  const RouteWs w = route_ws(B, H, N, d, block);
+  const fvattn_status wst = check_ws(route_workspace, workspace_bytes, w.total);
+  if (wst != FVATTN_OK) return wst;
+  auto base = static_cast<uint8_t*>(route_workspace);
+  auto hdr = reinterpret_cast<fvattn::WsHeader*>(base);
+  return from_cuda(fvattn::launch_order_lists(reinterpret_cast<const float*>(base + w.scores), B * H,
+                                              num_blocks(N, block), kv_idx, kv_cnt, &hdr->status,
+                                              static_cast<cudaStream_t>(stream)));
 }
 
 fvattn_status fvattn_sparse_fwd(const void* qp, const void* kp, const void* vp, void* op,

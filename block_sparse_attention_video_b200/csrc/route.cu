@@ -335,3 +335,73 @@ cudaError_t launch_select_topp(const float* rows_in, int BH, int nb, float p, in
 }
 
 }  // namespace fvattn
+
+namespace fvattn {
+
+// Descending order of (score, then lower block index) as one 64-bit key: the
+// float bits mapped to an unsigned order (negatives flipped), then the
+// complemented index.
+__device__ __forceinline__ unsigned long long importance_key(float s, int j) {
+  const uint32_t b = __float_as_uint(s);
+  const uint32_t o = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return (static_cast<unsigned long long>(o) << 32) | static_cast<unsigned long long>(0xFFFFFFFFu - j);
+}
+
+// One CTA per row: the row's cnt selected blocks sorted by descending score
+// (bitonic network in shared memory over the next power of two), written back
+// over the first cnt entries of the list.
+__global__ void __launch_bounds__(kRouteThreads)
+    order_lists_kernel(const float* __restrict__ S, int ld, int nb, int* __restrict__ kv_idx,
+                       const int* __restrict__ kv_cnt, int* status) {
+  extern __shared__ unsigned long long okeys[];
+  const int r = blockIdx.x;
+  const float* srow = S + static_cast<size_t>(r) * ld;
+  int* lst = kv_idx + static_cast<size_t>(r) * nb;
+  int cnt = kv_cnt[r];
+  if (cnt < 1 || cnt > nb) {
+    if (threadIdx.x == 0) record_status(status, FVATTN_ERR_INVALID_ARG);
+    cnt = min(max(cnt, 1), nb);
+  }
+  int n2 = 1;
+  while (n2 < cnt) n2 <<= 1;
+  for (int t = threadIdx.x; t < n2; t += blockDim.x) {
+    unsigned long long key = 0ull;     // pads sort last
+    if (t < cnt) {
+      int j = lst[t];
+      if (j < 0 || j >= nb) {
+        record_status(status, FVATTN_ERR_INVALID_ARG);
+        j = min(max(j, 0), nb - 1);
+      }
+      key = importance_key(srow[j], j);
+    }
+    okeys[t] = key;
+  }
+  for (int size = 2; size <= n2; size <<= 1)
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      __syncthreads();
+      for (int t = threadIdx.x; t < n2 / 2; t += blockDim.x) {
+        const int lo = 2 * t - (t & (stride - 1));
+        const int hi = lo + stride;
+        const bool desc = (lo & size) == 0;
+        const unsigned long long x = okeys[lo], y = okeys[hi];
+        if ((x < y) == desc) { okeys[lo] = y; okeys[hi] = x; }
+      }
+    }
+  __syncthreads();
+  for (int t = threadIdx.x; t < cnt; t += blockDim.x)
+    lst[t] = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(okeys[t] & 0xFFFFFFFFull));
+}
+
+cudaError_t launch_order_lists(const float* S, int BH, int nb, int* kv_idx, const int* kv_cnt, int* status,
+                               cudaStream_t st) {
+  int n2 = 1;
+  while (n2 < nb) n2 <<= 1;
+  const size_t smem = static_cast<size_t>(n2) * sizeof(unsigned long long);
+  cudaError_t e = cudaFuncSetAttribute(order_lists_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  order_lists_kernel<<<BH * nb, kRouteThreads, smem, st>>>(S, scores_ld(nb), nb, kv_idx, kv_cnt, status);
+  return cudaGetLastError();
+}
+
+}  // namespace fvattn

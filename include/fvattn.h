@@ -20,6 +20,11 @@
  *                                                        [FVAttn §2.1; GSRS §3.2, §A.1]
  *   fvattn_dense_fwd  the same kernel with every block selected (the dense
  *                     baseline every page compares against)
+ *   fvattn_order_lists_by_importance  optional: the routed lists in importance
+ *                     order (descending block score)     [FVAttn §3.1]
+ * Other entry points: fvattn_route_noalloc (routing for callers that cannot hand
+ * the library a workspace) and fvattn_wait_selftest (the kernels' bounded waits
+ * exercised without a fault).
  * Diagnostic of mask quality, from statistics the attention kernels record:
  *   fvattn_block_importance  exact block importance   [GSRS §5.3, §A.2, §A.3]
  *   fvattn_attention_recall  attention recall of a mask            [GSRS §3.2]
@@ -161,6 +166,21 @@ FVATTN_API fvattn_status fvattn_route(const void* q, const void* k, int B, int H
                            int k_min, void* qp_out, void* kp_out, int32_t* kv_idx,
                            int32_t* kv_cnt, int64_t* head_work, void* workspace,
                            size_t workspace_bytes, void* stream);
+
+/* Importance order of the routed lists [FVAttn §3.1: the routing front end
+ * yields a block-importance ranking, which slack augmentation consumes in
+ * order]: reorders the first kv_cnt[b,h,i] entries of every row of kv_idx, in
+ * place, by descending block score of the preceding fvattn_route call made
+ * with the same workspace (same B, H, N, d, block; the workspace still holds
+ * that call's block scores), ties in ascending block index. The set of each row
+ * is unchanged and the attention entry points accept either order (results
+ * agree up to fp32 rounding order). kv_idx [B,H,nb,nb] int32 in/out, kv_cnt
+ * [B,H,nb] int32 in. A count outside [1, nb] or an entry outside [0, nb) is
+ * clamped and recorded as FVATTN_ERR_INVALID_ARG in the route workspace's
+ * status word. Workspace: the route's (fvattn_workspace_bytes(FVATTN_OP_ROUTE, ...)). */
+FVATTN_API fvattn_status fvattn_order_lists_by_importance(int32_t* kv_idx, const int32_t* kv_cnt, int B, int H,
+                                                          int N, int d, int block, void* route_workspace,
+                                                          size_t workspace_bytes, void* stream);
 
 /* fvattn_route for callers that cannot allocate device memory at the call
  * site (an engine plugin with no scratch buffer to offer, or a hot loop where

@@ -291,3 +291,72 @@ def test_batch_of_two_tensor_core():
     op, _ = _attn_gpu(w, qp, kp, vp, kv_idx, kv_cnt)
     _check_attention(w, qp, kp, vp, op, mask, _sample_blocks(w, nb, cnt, per_head=4),
                      BF16_MAX_ABS, BF16_MEAN_ABS)
+
+
+def test_route_720p_bs64_sampled_heads():
+    """64-token blocks (1x8x8 tiles) at the 720p shape: every query block of 8 heads against
+    the oracle's routing (the rest of the heads are routed by the same launch)."""
+    w = S.WORKLOADS["wan14b-720p"].replace(name="wan14b-720p-bs64", block=64, tile=(1, 8, 8))
+    q, k, _ = S.make_qkv(w, device="cuda")
+    grid, qp, kp, kv_idx, kv_cnt, hw = _route_gpu(w, q, k)
+    heads = list(range(0, w.H, 5))
+    orc = O.route(_np(q[:, heads]), _np(k[:, heads]), w.grid6, w.block, w.p, w.k_min)
+    idx, cnt = kv_idx[:, heads].cpu().numpy(), kv_cnt[:, heads].cpu().numpy()
+    check_lists_valid(idx, cnt, grid.nb, w.k_min)
+    assert np.array_equal(hw.cpu().numpy(), kv_cnt.cpu().numpy().astype(np.int64).sum(-1))
+    assert_mask_parity(compare_masks(mask_from_lists(idx, cnt, grid.nb), orc, w.p), w.name)
+
+
+@pytest.mark.parametrize("w", [ODD128, S.WORKLOADS["wan1.3b-480p"], BS64], ids=lambda w: w.name)
+def test_lists_in_importance_order(w):
+    """The same sets as the routed lists, reordered by descending score: against the
+    oracle's scores every list is non-increasing up to the near-cut tolerance, and the
+    attention result does not change beyond rounding."""
+    q, k, v = S.make_qkv(w, device="cuda")
+    grid = F.Grid.make(w.grid, w.tile, w.block)
+    nb, npad = grid.nb, grid.nb * w.block
+    dev = q.device
+    qp = torch.empty((w.B, w.H, npad, w.d), dtype=q.dtype, device=dev)
+    kp = torch.empty_like(qp)
+    kv_idx = torch.empty((w.B, w.H, nb, nb), dtype=torch.int32, device=dev)
+    kv_cnt = torch.empty((w.B, w.H, nb), dtype=torch.int32, device=dev)
+    hw = torch.empty((w.B, w.H), dtype=torch.int64, device=dev)
+    ws = F.alloc_workspace(F.fvattn_workspace_bytes(F.FVATTN_OP_ROUTE, w.B, w.H, w.N, w.d, w.block), dev)
+    F.fvattn_route(q, k, grid, w.p, w.k_min, kv_idx, kv_cnt, hw, ws, qp_out=qp, kp_out=kp)
+    asc = kv_idx.clone()
+    F.fvattn_order_lists_by_importance(kv_idx, kv_cnt, w.N, w.d, w.block, ws)
+    assert F.fvattn_workspace_status(ws) == F.FVATTN_OK
+    orc = O.route(_np(q), _np(k), w.grid6, w.block, w.p, w.k_min)
+    idx, cnt, idx_asc = kv_idx.cpu().numpy(), kv_cnt.cpu().numpy(), asc.cpu().numpy()
+    for row in np.ndindex(*cnt.shape):
+        c = int(cnt[row])
+        got = idx[row][:c]
+        assert np.array_equal(np.sort(got), idx_asc[row][:c]), row
+        # the GPU orders by its fp32 logits; scores closer than their rounding may swap
+        s = orc["scores"][row][got]
+        assert np.all(s[1:] <= s[:-1] * (1 + 1e-4)), (row, s[:8])
+    vp = torch.empty_like(qp)
+    F.fvattn_permute(v, vp, grid)
+    a, _ = _attn_gpu(w, qp, kp, vp, asc, kv_cnt)
+    b, _ = _attn_gpu(w, qp, kp, vp, kv_idx, kv_cnt)
+    d = (a.float() - b.float()).abs()[:, :, : w.N]
+    assert float(d.max()) <= 2e-2
+
+
+def test_importance_order_breaks_ties_by_block_index():
+    # q = 0: every score of a row is equal, so the order is ascending block index
+    w = ODD128.replace(p=0.5, k_min=1)
+    _, k, _ = S.make_qkv(w, device="cuda")
+    q = torch.zeros_like(k)
+    grid = F.Grid.make(w.grid, w.tile, w.block)
+    nb = grid.nb
+    kv_idx = torch.empty((w.B, w.H, nb, nb), dtype=torch.int32, device="cuda")
+    kv_cnt = torch.empty((w.B, w.H, nb), dtype=torch.int32, device="cuda")
+    hw = torch.empty((w.B, w.H), dtype=torch.int64, device="cuda")
+    ws = F.alloc_workspace(F.fvattn_workspace_bytes(F.FVATTN_OP_ROUTE, w.B, w.H, w.N, w.d, w.block), "cuda")
+    F.fvattn_route(q, k, grid, w.p, w.k_min, kv_idx, kv_cnt, hw, ws)
+    asc = kv_idx.clone()
+    F.fvattn_order_lists_by_importance(kv_idx, kv_cnt, w.N, w.d, w.block, ws)
+    assert F.fvattn_workspace_status(ws) == F.FVATTN_OK
+    c = int(kv_cnt.min())
+    assert torch.equal(kv_idx[..., :c], asc[..., :c])
