@@ -51,8 +51,8 @@ METRIC = "sparse attn ms/call & effective TFLOP/s (Wan-14B 720p shape) vs own de
 # head's K and V) fits in L2 at both sizes, so the re-read factor carries over.
 # After any change of the source the traffic is unknown and reported as null.
 ATTN_TRAFFIC = {
-    # 1,021,980,416 read + 320,834,816 written; Q, K, V, O at 2 B x 40 x 256 x 128 x 128
-    "bf16": {"bytes_480p": 1021980416 + 320834816, "algorithmic_480p": 4 * 40 * 256 * 128 * 128 * 2,
+    # 1,022,458,880 read + 320,556,288 written; Q, K, V, O at 2 B x 40 x 256 x 128 x 128
+    "bf16": {"bytes_480p": 1022458880 + 320556288, "algorithmic_480p": 4 * 40 * 256 * 128 * 128 * 2,
              "src": "75a9d8b8ec84c740"},
     # 847,159,296 read + 316,532,224 written; Q, K, O at 2 B and the E4M3 V at 1 B
     "fp8v": {"bytes_480p": 847159296 + 316532224, "algorithmic_480p": 7 * 40 * 256 * 128 * 128,
