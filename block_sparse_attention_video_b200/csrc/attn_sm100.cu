@@ -19,7 +19,8 @@
 //   warps 4-7  softmax / epilogue of slot 1
 //   warp  8    TMA producer (one elected thread); claims work units from a
 //              global counter and publishes them to the other roles
-//   warp  9    TMEM allocator and MMA issuer (one elected thread)
+//   warp  9    TMEM allocator and MMA issuer (the whole warp walks the unit;
+//              one elected lane issues each MMA and commit)
 //   warps 10-11 idle
 // The block launches with 168 registers per thread (384 x 168 = 64,512); the
 // third warpgroup drops to 128 and the two softmax warpgroups rise to 184
@@ -67,6 +68,7 @@
 
 namespace fvattn {
 namespace sm100 {
+
 
 constexpr int kUnitRows = 256;
 constexpr int kQHalfBytes = 128 * 128;      // 16 KB: 128 rows x 64 columns (128 bytes)
@@ -323,88 +325,97 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_plain(&sm.kv_full[o % kStages], (o / kStages) & 1);
       for (int X = 0; X < 2; ++X)
         if (qn[X] > 0) mbar_wait_plain(&sm.q_full[X], (qn[X] - 1) & 1);
-    } else if (warp == 9 && lane == 0) {
+    } else if (warp == 9) {
       // ---------------------------------------------------------- MMA issuer
+      // The whole warp runs this loop: every value in it is warp-uniform, each wait
+      // is a warp vote, and one elected lane issues each tcgen05.mma / commit. The
+      // shared-memory descriptors are built once; a stage or K slice is a constant
+      // added to the start-address field (addresses stay inside the 18-bit window,
+      // so the field never carries).
       int base = 0, un = 0;
       int qn[2] = {0, 0};
       int pn[2] = {0, 0};
-      const uint32_t q_addr[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
-      const uint32_t kv_addr = smem_u32(sm.kv);
+      const uint64_t dq[2] = {umma_desc_sw128(smem_u32(sm.q[0]), 16, 1024),
+                              umma_desc_sw128(smem_u32(sm.q[1]), 16, 1024)};
+      const uint64_t dk = umma_desc_sw128(smem_u32(sm.kv), 16, 1024);
+      const uint64_t dv = umma_desc_sw128(smem_u32(sm.kv), T::kKVHalf, 1024);
+      auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, P.status));
+      };
       bool ok = true;
       while (ok) {
         const int b = un & 1;
-        if (!mbar_wait(&sm.unit_full[b], (un >> 1) & 1, abort_flag, P.status)) break;
+        if (!wait(&sm.unit_full[b], (un >> 1) & 1)) break;
         const int u = *reinterpret_cast<volatile int*>(&sm.unit_box[b]);
-        mbar_arrive(&sm.unit_empty[b]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.unit_empty[b]);
         ++un;
         const Unit x = decode_unit<BN>(u, P);
         if (x.cnt == 0) break;
         const int cnt = (x.cnt + T::kBPS - 1) / T::kBPS;   // steps of 128 keys
-        auto kv_ready = [&](int o) -> bool {
-          return mbar_wait(&sm.kv_full[o % kStages], (o / kStages) & 1, abort_flag, P.status);
-        };
+        auto kv_ready = [&](int o) -> bool { return wait(&sm.kv_full[o % kStages], (o / kStages) & 1); };
         auto s_op = [&](int X, int k) -> bool {   // S_X = Q_X K(k)^T, K(k) already waited on
           if (k == 0) {
-            if (!mbar_wait(&sm.q_full[X], qn[X] & 1, abort_flag, P.status)) return false;
+            if (!wait(&sm.q_full[X], qn[X] & 1)) return false;
             ++qn[X];
           }
           tc_fence_after();
-          const uint32_t ka = kv_addr + ((base + 2 * k) % kStages) * T::kKVBytes;
+          const uint64_t ks = dk + static_cast<uint64_t>(((base + 2 * k) % kStages) * (T::kKVBytes >> 4));
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
-            umma_ss(tmem + X * 128,
-                    umma_desc_sw128(q_addr[X] + (kk >> 2) * kQHalfBytes + (kk & 3) * 32, 16, 1024),
-                    umma_desc_sw128(ka + (kk >> 2) * T::kKVHalf + (kk & 3) * 32, 16, 1024),
-                    T::kIdescQK, kk > 0 ? 1u : 0u);
+            constexpr int kQH = kQHalfBytes;
+            const uint32_t qo = ((kk >> 2) * kQH + (kk & 3) * 32) >> 4;
+            const uint32_t ko = ((kk >> 2) * T::kKVHalf + (kk & 3) * 32) >> 4;
+            umma_ss_elect(tmem + X * 128, dq[X] + qo, ks + ko, T::kIdescQK, kk > 0 ? 1u : 0u);
           }
-          umma_commit(&sm.s_full[X]);
-          if (k == cnt - 1) umma_commit(&sm.q_empty[X]);
+          umma_commit_elect(&sm.s_full[X]);
+          if (k == cnt - 1) umma_commit_elect(&sm.q_empty[X]);
           return true;
         };
         auto pv_op = [&](int X, int k) -> bool {  // O_X += P_X V(k), V(k) already waited on
           // P arrives in two halves (key columns [0, 64) and [64, 128)); the
           // first half's MMAs run while the softmax warps finish the second.
-          const uint32_t va = kv_addr + ((base + 2 * k + 1) % kStages) * T::kKVBytes;
+          const uint64_t vs = dv + static_cast<uint64_t>(((base + 2 * k + 1) % kStages) * (T::kKVBytes >> 4));
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            if (!mbar_wait(&sm.p_full[X][h], pn[X] & 1, abort_flag, P.status)) return false;
+            if (!wait(&sm.p_full[X][h], pn[X] & 1)) return false;
             tc_fence_after();
             constexpr int kPerHalf = T::kStepKeys / 2 / T::kPVK;
 #pragma unroll
             for (int kk = h * kPerHalf; kk < (h + 1) * kPerHalf; ++kk) {
               // kk-th K slice of P: 8 TMEM columns (16 bf16 or 32 E4M3 keys); of V:
               // kPVK rows of 128 bytes
-              const uint64_t bd = umma_desc_sw128(va + kk * T::kPVK * 128, T::kKVHalf, 1024);
+              const uint64_t bd = vs + static_cast<uint32_t>((kk * T::kPVK * 128) >> 4);
               if constexpr (F8)
-                umma_ts_f8(tmem + 256 + X * 128, tmem + X * 128 + kk * 8, bd, T::kIdescPV,
-                           (k > 0 || kk > 0) ? 1u : 0u);
+                umma_ts_f8_elect(tmem + 256 + X * 128, tmem + X * 128 + kk * 8, bd, T::kIdescPV,
+                                 (k > 0 || kk > 0) ? 1u : 0u);
               else
-                umma_ts(tmem + 256 + X * 128, tmem + X * 128 + kk * 8, bd, T::kIdescPV,
-                        (k > 0 || kk > 0) ? 1u : 0u);
+                umma_ts_elect(tmem + 256 + X * 128, tmem + X * 128 + kk * 8, bd, T::kIdescPV,
+                              (k > 0 || kk > 0) ? 1u : 0u);
             }
           }
           ++pn[X];
-          if (k == cnt - 1) umma_commit(&sm.o_full[X]);
+          if (k == cnt - 1) umma_commit_elect(&sm.o_full[X]);
           return true;
         };
         const bool two = x.slot[1];
         ok = kv_ready(base) && s_op(0, 0) && (!two || s_op(1, 0));
-        if (ok) umma_commit(&sm.kv_empty[base % kStages]);
+        if (ok) umma_commit_elect(&sm.kv_empty[base % kStages]);
         for (int k = 1; ok && k < cnt; ++k) {
           ok = kv_ready(base + 2 * k - 1) && pv_op(0, k - 1) && kv_ready(base + 2 * k) && s_op(0, k) &&
                (!two || pv_op(1, k - 1));
           if (!ok) break;
-          umma_commit(&sm.kv_empty[(base + 2 * k - 1) % kStages]);
+          umma_commit_elect(&sm.kv_empty[(base + 2 * k - 1) % kStages]);
           ok = !two || s_op(1, k);
           if (!ok) break;
-          umma_commit(&sm.kv_empty[(base + 2 * k) % kStages]);
+          umma_commit_elect(&sm.kv_empty[(base + 2 * k) % kStages]);
         }
         if (ok) ok = kv_ready(base + 2 * cnt - 1) && pv_op(0, cnt - 1) && (!two || pv_op(1, cnt - 1));
-        if (ok) umma_commit(&sm.kv_empty[(base + 2 * cnt - 1) % kStages]);
+        if (ok) umma_commit_elect(&sm.kv_empty[(base + 2 * cnt - 1) % kStages]);
         base += 2 * cnt;
       }
-      // Drain: every MMA this thread issued has completed before TMEM is freed.
-      umma_commit(&sm.mma_done);
+      // Drain: every MMA this warp issued has completed before TMEM is freed.
+      umma_commit_elect(&sm.mma_done);
       mbar_wait_plain(&sm.mma_done, 0);
     }
     teardown();
