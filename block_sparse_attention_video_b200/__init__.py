@@ -61,7 +61,7 @@ EXPORTED = ("fvattn_workspace_bytes", "fvattn_permute", "fvattn_route", "fvattn_
             "fvattn_sparse_fwd", "fvattn_dense_fwd", "fvattn_block_importance", "fvattn_attention_recall",
             "fvattn_select_topp", "fvattn_lvsa_lists", "fvattn_hilbert_table", "fvattn_quantize_v",
             "fvattn_sparse_fwd_fp8v", "fvattn_dense_fwd_fp8v",
-            "fvattn_workspace_status", "fvattn_status_string", "fvattn_wait_selftest", "fvattn_exp2_selftest",
+            "fvattn_workspace_status", "fvattn_status_string", "fvattn_wait_selftest",
             "fvattn_permute_quantize_v", "fvattn_order_lists_by_importance")
 
 
@@ -144,8 +144,6 @@ _lib.fvattn_workspace_status.argtypes = [_c_void_p, _c_void_p]
 _lib.fvattn_workspace_status.restype = _c_int
 _lib.fvattn_wait_selftest.argtypes = [_c_void_p, _c_void_p, _c_size_t, _c_void_p]
 _lib.fvattn_wait_selftest.restype = _c_int
-_lib.fvattn_exp2_selftest.argtypes = [_c_void_p, ctypes.c_int64, _c_void_p, _c_void_p, _c_void_p]
-_lib.fvattn_exp2_selftest.restype = _c_int
 _lib.fvattn_status_string.argtypes = [_c_int]
 _lib.fvattn_status_string.restype = ctypes.c_char_p
 
@@ -536,19 +534,6 @@ def fvattn_wait_selftest(results, workspace, stream=None):
     _check(_call(dev, _lib.fvattn_wait_selftest, _ptr(results), _ptr(workspace),
                  workspace.numel() * workspace.element_size(), _stream(stream, dev)), "fvattn_wait_selftest")
     return results
-
-
-def fvattn_exp2_selftest(x, y_fma, y_mufu, stream=None):
-    """The softmax's two forms of 2^x on x [n] fp32 (device): y_fma (FMA-pipe
-    polynomial) and y_mufu (ex2.approx), both [n] fp32 on x's device."""
-    _need_cuda(x, y_fma, y_mufu)
-    dev = x.device
-    n = x.numel()
-    for t, name in ((x, "x"), (y_fma, "y_fma"), (y_mufu, "y_mufu")):
-        _expect(t, name, dev, (n,), torch.float32)
-    _check(_call(dev, _lib.fvattn_exp2_selftest, _ptr(x), n, _ptr(y_fma), _ptr(y_mufu),
-                 _stream(stream, dev)), "fvattn_exp2_selftest")
-    return y_fma, y_mufu
 
 
 def alloc_workspace(nbytes: int, device) -> torch.Tensor:

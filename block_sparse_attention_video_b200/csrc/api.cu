@@ -46,8 +46,6 @@ cudaError_t launch_quantize_v(const void* v, int BH, int N, int npad, uint8_t* v
                               unsigned int* amax_bits, cudaStream_t st);
 size_t vquant_ws_bytes(int BH);
 cudaError_t launch_wait_selftest(long long* out, int* status, cudaStream_t st);
-cudaError_t launch_exp2_selftest(const float* x, long long n, float* y_fma, float* y_mufu,
-                                 cudaStream_t st);
 cudaError_t launch_order_lists(const float* S, int BH, int nb, int* kv_idx, const int* kv_cnt, int* status,
                                cudaStream_t st);
 cudaError_t launch_permute_quantize_v(const void* v, int BH, int N, int bs, const TileGeom& g, uint8_t* vq,
@@ -560,16 +558,6 @@ fvattn_status fvattn_wait_selftest(int64_t* results, void* workspace, size_t wor
   if (cudaMemsetAsync(workspace, 0, kWsHeaderBytes, st) != cudaSuccess) return FVATTN_ERR_CUDA;
   if (cudaMemsetAsync(results, 0, 8 * sizeof(int64_t), st) != cudaSuccess) return FVATTN_ERR_CUDA;
   return from_cuda(fvattn::launch_wait_selftest(reinterpret_cast<long long*>(results), &hdr->status, st));
-}
-
-fvattn_status fvattn_exp2_selftest(const float* x, int64_t n, float* y_fma, float* y_mufu,
-                                   void* stream) {
-  if (n < 0 || n > (int64_t(1) << 31)) return FVATTN_ERR_INVALID_ARG;
-  if (n == 0) return FVATTN_OK;
-  if (!x || !y_fma || !y_mufu || !aligned(x, 4) || !aligned(y_fma, 4) || !aligned(y_mufu, 4))
-    return FVATTN_ERR_INVALID_ARG;
-  return from_cuda(fvattn::launch_exp2_selftest(x, static_cast<long long>(n), y_fma, y_mufu,
-                                                static_cast<cudaStream_t>(stream)));
 }
 
 fvattn_status fvattn_workspace_status(const void* workspace, void* stream) {

@@ -50,12 +50,6 @@
 // Softmax: exponent base 2 with scale*log2(e) folded in, P rounded to bf16,
 // fp32 row sums. The running max is only raised (and O rescaled in TMEM) when a
 // block's max exceeds it by more than 8 (a factor 256), which keeps P <= 256.
-// MUFU delivers 16 exponentials per clock per SM, as many as the tensor pipe
-// needs for both tiles at full rate, so on one-block steps (128-token blocks)
-// three pairs in eight are taken on the FMA pipe instead (ex2_pair_fma: a cubic
-// polynomial, relative error below 1e-4, far under P's own bf16 rounding; a key
-// masked past N gets 2^-125 there instead of 0, which the fp32 sums do not resolve
-// and which multiplies a zero row of V).
 //
 // 8-bit V variant (F8 = true) [FVAttn §3.4: V is quantized on the GPU before
 // attention]: V arrives as E4M3 codes [B*H, Npad, 128] with one fp32 scale per
@@ -594,24 +588,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             // a half the row does not attend (two entries per step): every x = -inf, so P = 0
             const float2 negc =
                 (BPS == 1 || mem[c / CPE]) ? negm : make_float2(-INFINITY, -INFINITY);
-            // the FMA-pipe pairs take y = sat(x / 256 + 125 / 256) = sat(s * cy + cb)
-            const float cy = sl2 * (1.f / 256.f);
-            const float cb = negc.x * (1.f / 256.f) + 125.f / 256.f;
             __half2 hs[2] = {__float2half2_rn(0.f), __float2half2_rn(0.f)};
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              float p0, p1;
-              if (BPS == 1 && (i % 8 == 2 || i % 8 == 5 || i % 8 == 7)) {   // compile-time: 3 pairs in 8 on the FMA pipe
-                const float2 pp = ex2_pair_fma(fma_sat(__uint_as_float(s[c][2 * i]), cy, cb),
-                                               fma_sat(__uint_as_float(s[c][2 * i + 1]), cy, cb));
-                p0 = pp.x;
-                p1 = pp.y;
-              } else {
-                const float2 xv = __ffma2_rn(
-                    make_float2(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])), sl2x2, negc);
-                p0 = ex2_approx(xv.x);
-                p1 = ex2_approx(xv.y);
-              }
+              const float2 xv = __ffma2_rn(
+                  make_float2(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])), sl2x2, negc);
+              const float p0 = ex2_approx(xv.x);
+              const float p1 = ex2_approx(xv.y);
               if constexpr (F8) {
                 // four keys per 32-bit word, lowest key in the low byte
                 const uint32_t q8 = pack_e4m3x2(p0, p1);

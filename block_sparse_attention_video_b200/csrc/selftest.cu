@@ -8,12 +8,7 @@
 // other waiter of the CTA return at once, and records FVATTN_ERR_TIMEOUT in the
 // workspace status word, so the kernel ends and the host reads the status.
 //
-// exp2_selftest_kernel evaluates the two forms of 2^x the attention softmax
-// uses, with the softmax's own argument transforms, so a test can hold them to
-// their error bounds: the MUFU form (ex2.approx on x) and the FMA-pipe form
-// (ex2_pair_fma on y = sat(x / 256 + 125 / 256), a saturating FMA as in the kernel).
-//
-// The wait self-test runs exactly those helpers on mbarriers that nothing ever arrives
+// This kernel runs exactly those helpers on mbarriers that nothing ever arrives
 // at: one thread waits until the limit runs out, a thread of another warp waits
 // on a second such barrier and is released by the abort flag, and the drain-style
 // wait (no abort flag) runs out too. It touches no TMA, tensor memory or global
@@ -61,32 +56,6 @@ __global__ void __launch_bounds__(64, 1) wait_selftest_kernel(long long* out, in
 
 cudaError_t launch_wait_selftest(long long* out, int* status, cudaStream_t st) {
   wait_selftest_kernel<<<1, 64, 0, st>>>(out, status);
-  return cudaGetLastError();
-}
-
-__global__ void __launch_bounds__(256) exp2_selftest_kernel(const float* __restrict__ x, long long n,
-                                                             float* __restrict__ y_fma,
-                                                             float* __restrict__ y_mufu) {
-  const long long i = 2 * (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x);
-  if (i >= n) return;
-  const float x0 = x[i];
-  const float x1 = i + 1 < n ? x[i + 1] : 0.f;
-  const float2 p = ex2_pair_fma(fma_sat(x0, 1.f / 256.f, 125.f / 256.f),
-                                fma_sat(x1, 1.f / 256.f, 125.f / 256.f));
-  y_fma[i] = p.x;
-  y_mufu[i] = ex2_approx(x0);
-  if (i + 1 < n) {
-    y_fma[i + 1] = p.y;
-    y_mufu[i + 1] = ex2_approx(x1);
-  }
-}
-
-cudaError_t launch_exp2_selftest(const float* x, long long n, float* y_fma, float* y_mufu,
-                                 cudaStream_t st) {
-  if (n <= 0) return cudaSuccess;
-  const long long pairs = (n + 1) / 2;
-  const unsigned grid = static_cast<unsigned>((pairs + 255) / 256);
-  exp2_selftest_kernel<<<grid, 256, 0, st>>>(x, n, y_fma, y_mufu);
   return cudaGetLastError();
 }
 

@@ -277,35 +277,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x for a pair of values on the FMA pipe (no MUFU), for x <= 131; values below
-// -125 give 2^-125. The caller passes y = sat(x / 256 + 125 / 256) (a saturating
-// FMA, so x is clamped to [-125, 131] without an integer min/max). Cody-Waite style
-// reduction: t = 256 y + (1.5 * 2^23 - 125) rounds x to an integer n held in t's low
-// mantissa bits; f = x - n lies in [-1/2, 1/2]; 2^f comes from a cubic minimax
-// polynomial (our own Remez fit on [-1/2, 1/2], relative error below 1e-4); 2^n
-// enters as n << 23 added to the bit pattern (t's bits shifted left by 23 leave
-// exactly n << 23, the constant part of t shifting out).
-__device__ __forceinline__ float2 ex2_pair_fma(float y0, float y1) {
-  constexpr float kM = 12582912.0f - 125.0f;
-  constexpr float kC0 = 0.99992806f, kC1 = 0.69326097f, kC2 = 0.24261113f, kC3 = 0.05517167f;
-  const float2 y = make_float2(y0, y1);
-  const float2 t = __ffma2_rn(y, make_float2(256.f, 256.f), make_float2(kM, kM));
-  const float2 w = __fadd2_rn(make_float2(kM, kM), make_float2(-t.x, -t.y));
-  const float2 f = __ffma2_rn(y, make_float2(256.f, 256.f), w);
-  float2 q = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
-  q = __ffma2_rn(q, f, make_float2(kC1, kC1));
-  q = __ffma2_rn(q, f, make_float2(kC0, kC0));
-  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
-}
-
-// a * b + c rounded once and clamped to [0, 1]
-__device__ __forceinline__ float fma_sat(float a, float b, float c) {
-  float r;
-  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
 // Two fp32 values to E4M3 (round to nearest even, saturating at +-448); lo in
 // the low byte.
 __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {

@@ -23,9 +23,8 @@
  *   fvattn_order_lists_by_importance  optional: the routed lists in importance
  *                     order (descending block score)     [FVAttn §3.1]
  * Other entry points: fvattn_route_noalloc (routing for callers that cannot hand
- * the library a workspace), fvattn_wait_selftest (the kernels' bounded waits
- * exercised without a fault) and fvattn_exp2_selftest (the softmax's two forms
- * of 2^x, for tests of their error bounds).
+ * the library a workspace) and fvattn_wait_selftest (the kernels' bounded waits
+ * exercised without a fault).
  * Diagnostic of mask quality, from statistics the attention kernels record:
  *   fvattn_block_importance  exact block importance   [GSRS §5.3, §A.2, §A.3]
  *   fvattn_attention_recall  attention recall of a mask            [GSRS §3.2]
@@ -405,19 +404,6 @@ FVATTN_API fvattn_status fvattn_workspace_status(const void* workspace, void* st
  * Workspace: 256 bytes, 256-byte aligned (fvattn_workspace_bytes of
  * FVATTN_OP_DENSE_FWD gives that size). Returns FVATTN_OK once launched. */
 FVATTN_API fvattn_status fvattn_wait_selftest(int64_t* results, void* workspace, size_t workspace_bytes,
-                                              void* stream);
-
-/* The two forms of 2^x the attention softmax uses [GSRS §A.1: the online softmax's
- * exponentials], evaluated one per input so that a test can hold them to their
- * bounds (this library's own check, not a step of the path):
- *   y_mufu[i] = ex2.approx.ftz.f32(x[i])  (the MUFU form, 5 pairs in 8);
- *   y_fma[i]  = the FMA-pipe form (3 pairs in 8 on one-block steps): y =
- *               sat(x/256 + 125/256) by one saturating FMA, then Cody-Waite
- *               reduction and a cubic minimax polynomial; relative error below 1e-4
- *               for -125 <= x <= 131, 2^-125 for x below -125.
- * x, y_fma, y_mufu: [n] fp32, device, 4-byte aligned; 0 <= n <= 2^31 (n = 0: nothing).
- * Errors: FVATTN_ERR_INVALID_ARG for null or misaligned pointers or n out of range. */
-FVATTN_API fvattn_status fvattn_exp2_selftest(const float* x, int64_t n, float* y_fma, float* y_mufu,
                                               void* stream);
 
 /* Static string for a status code (never NULL). */

@@ -66,14 +66,6 @@ int main(void) {
     CHECK(st == FVATTN_ERR_INVALID_ARG, 37);
     st = fvattn_wait_selftest((int64_t*)0x100000, NULL, 0, NULL);
     CHECK(st == FVATTN_ERR_WORKSPACE, 38);
-    /* the exponential self-test: null outputs and a negative count are rejected,
-       and an empty input launches nothing */
-    st = fvattn_exp2_selftest((const float*)0x100000, 16, NULL, (float*)0x200000, NULL);
-    CHECK(st == FVATTN_ERR_INVALID_ARG, 39);
-    st = fvattn_exp2_selftest((const float*)0x100000, -1, (float*)0x200000, (float*)0x300000, NULL);
-    CHECK(st == FVATTN_ERR_INVALID_ARG, 46);
-    st = fvattn_exp2_selftest(NULL, 0, NULL, NULL, NULL);
-    CHECK(st == FVATTN_OK, 47);
   }
   {
     int s;
