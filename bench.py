@@ -61,6 +61,19 @@ ATTN_TRAFFIC = {
 ATTN_SRC = os.path.join(ROOT, "block_sparse_attention_video_b200", "csrc", "attn_sm100.cu")
 
 
+# A 128 x 256 x 16 bf16 tcgen05.mma (kind::f16, fp32 accumulate) takes 128 SM cycles:
+# 8,192 FLOP per clock per SM on the tensor pipe.
+TENSOR_BF16_FLOP_PER_CLK_SM = 8192
+
+
+def _frac_at_clock(achieved_tflops: float, clocks, dev):
+    if not clocks or not clocks.get("sm_mhz"):
+        return None
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    peak = TENSOR_BF16_FLOP_PER_CLK_SM * sms * clocks["sm_mhz"] * 1e6 / 1e12
+    return achieved_tflops / peak
+
+
 def _attn_traffic(kind: str, algorithmic_bytes: float):
     """(scaled DRAM bytes per launch, note) for the current kernel source, or (None, why)."""
     import hashlib
@@ -648,6 +661,10 @@ def run_fvattn(args):
                      "peak": pk["bf16_sus"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_sus"],
                      "peak_kind": f"{pk['source']} bf16 sustained (kernel timed inside a long step)",
                      "frac_of_burst_peak": achieved / pk["bf16"],
+                     "frac_at_clock": _frac_at_clock(achieved, clocks, dev),
+                     "frac_at_clock_note": "achieved / (8,192 bf16 FLOP per clock per SM x SMs x the median SM "
+                                           "clock sampled in the timed region): the kernel's share of what the "
+                                           "tensor pipes deliver at the clock it actually ran at",
                      "traffic": traffic_bf16, "traffic_note": traffic_bf16_note,
                      "traffic_unit": "bytes per launch (DRAM read + write)",
                      "algorithmic_bytes": attn_alg_bytes},
