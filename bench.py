@@ -283,7 +283,7 @@ def oracle_check(w, qn, kn, vn, idx, cnt, op_perm, heads, per_head, rng, budget_
 
 LVSA_WINDOW, LVSA_PERIOD, LVSA_STEP = 2, 8, 0
 GSRS_SEARCH_P = 0.9
-E2E_HEAD_GROUPS = 4
+E2E_HEAD_GROUPS = 10
 
 
 def _median_ms(fn, stream, warmup, reps):
