@@ -15,7 +15,7 @@ if torch.cuda.is_available():
     import block_sparse_attention_video_b200 as F
 
 
-@pytest.mark.parametrize("head_groups", [1, 3])
+@pytest.mark.parametrize("head_groups", [1, 3, 12])   # 12: one head per range
 @pytest.mark.parametrize("dense", [False, True])
 def test_host_pipeline_matches_per_call_results(dense, head_groups):
     w = S.WORKLOADS["wan1.3b-480p"]
