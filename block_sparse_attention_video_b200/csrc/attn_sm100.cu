@@ -354,8 +354,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (x.cnt == 0) break;
         const int cnt = (x.cnt + T::kBPS - 1) / T::kBPS;   // steps of 128 keys
         auto kv_ready = [&](int o) -> bool { return wait(&sm.kv_full[o % kStages], (o / kStages) & 1); };
+        // Member-only MMAs with 64-token blocks: a unit there spans four query blocks,
+        // and slot X computes S and P.V for a step only when one of its two query
+        // blocks selected one of the step's entries (the softmax warps skip the same
+        // steps, decided from the same entries). Per 32 union entries one coalesced
+        // load and two ballots give each entry's slot membership; the next window's
+        // entries are loaded ahead. With 128-token blocks every slot computes every
+        // step: there a skip saves less than the test costs in this warp.
+        constexpr int G = T::kGroup;
+        constexpr uint32_t kMask0 = (1u << (G / 2)) - 1u, kMask1 = kMask0 << (G / 2);
+        uint32_t win[2] = {~0u, ~0u}, prev[2] = {~0u, ~0u};
+        int wbase = 0;
+        uint32_t ent_next = (BN == 64 && x.list && lane < x.cnt) ? __ldg(x.list + lane) : 0u;
+        auto refill = [&]() {
+          prev[0] = win[0];
+          prev[1] = win[1];
+          win[0] = __ballot_sync(0xffffffffu, ((ent_next >> 16) & kMask0) != 0u);
+          win[1] = __ballot_sync(0xffffffffu, ((ent_next >> 16) & kMask1) != 0u);
+          const int nx = wbase + 32 + lane;
+          ent_next = (x.list && nx < x.cnt) ? __ldg(x.list + nx) : 0u;
+        };
+        if (BN == 64 && x.list) refill();
+        // Steps are asked for in the order k-1, k (slot 0), k-1, k (slot 1): never more
+        // than one step behind the newest, so the previous window covers the older one.
+        auto member = [&](int X, int k) -> bool {
+          if (BN != 64 || !x.list) return true;
+          const int e0 = k * T::kBPS;
+          while (e0 >= wbase + 32) {
+            wbase += 32;
+            refill();
+          }
+          const uint32_t w = e0 >= wbase ? win[X] : prev[X];
+          const int sh = e0 >= wbase ? e0 - wbase : e0 - wbase + 32;
+          return ((w >> sh) & ((1u << T::kBPS) - 1u)) != 0u;
+        };
+        bool started[2] = {false, false};
         auto s_op = [&](int X, int k) -> bool {   // S_X = Q_X K(k)^T, K(k) already waited on
-          if (k == 0) {
+          if (!member(X, k)) return true;
+          if (!started[X]) {
             if (!wait(&sm.q_full[X], qn[X] & 1)) return false;
             ++qn[X];
           }
@@ -369,12 +405,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_ss_elect(tmem + X * 128, dq[X] + qo, ks + ko, T::kIdescQK, kk > 0 ? 1u : 0u);
           }
           umma_commit_elect(&sm.s_full[X]);
-          if (k == cnt - 1) umma_commit_elect(&sm.q_empty[X]);
+          started[X] = true;
           return true;
         };
+        bool pv_started[2] = {false, false};
         auto pv_op = [&](int X, int k) -> bool {  // O_X += P_X V(k), V(k) already waited on
           // P arrives in two halves (key columns [0, 64) and [64, 128)); the
           // first half's MMAs run while the softmax warps finish the second.
+          if (!member(X, k)) return true;
           const uint64_t vs = dv + static_cast<uint64_t>(((base + 2 * k + 1) % kStages) * (T::kKVBytes >> 4));
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -388,14 +426,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint64_t bd = vs + static_cast<uint32_t>((kk * T::kPVK * 128) >> 4);
               if constexpr (F8)
                 umma_ts_f8_elect(tmem + 256 + X * 128, tmem + X * 128 + kk * 8, bd, T::kIdescPV,
-                                 (k > 0 || kk > 0) ? 1u : 0u);
+                                 (pv_started[X] || kk > 0) ? 1u : 0u);
               else
                 umma_ts_elect(tmem + 256 + X * 128, tmem + X * 128 + kk * 8, bd, T::kIdescPV,
-                              (k > 0 || kk > 0) ? 1u : 0u);
+                              (pv_started[X] || kk > 0) ? 1u : 0u);
             }
           }
           ++pn[X];
-          if (k == cnt - 1) umma_commit_elect(&sm.o_full[X]);
+          pv_started[X] = true;
           return true;
         };
         const bool two = x.slot[1];
@@ -412,6 +450,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ok) ok = kv_ready(base + 2 * cnt - 1) && pv_op(0, cnt - 1) && (!two || pv_op(1, cnt - 1));
         if (ok) umma_commit_elect(&sm.kv_empty[(base + 2 * cnt - 1) % kStages]);
+        if (ok) {
+          // Q and O of both slots are released once every MMA of the unit is done.
+          // (A slot always has a member step: each query block selects at least one
+          // key block. Should one have none, its Q phase is still consumed here.)
+          for (int X = 0; X < (two ? 2 : 1); ++X) {
+            if (!started[X]) {
+              if (!wait(&sm.q_full[X], qn[X] & 1)) break;
+              ++qn[X];
+            }
+            umma_commit_elect(&sm.q_empty[X]);
+            umma_commit_elect(&sm.o_full[X]);
+          }
+        }
         base += 2 * cnt;
       }
       // Drain: every MMA this warp issued has completed before TMEM is freed.
@@ -432,6 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const int qb = (X * 128 + row) / BN;  // query block of this row within the unit
+    const uint32_t kSlotMask = ((1u << (T::kGroup / 2)) - 1u) << (X * (T::kGroup / 2));   // this slot's member bits
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tS = tmem + lane_off + X * 128;
     const uint32_t tO = tmem + lane_off + 256 + X * 128;
@@ -461,12 +513,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int h = 0; h < BPS; ++h) e_next[h] = h < x.cnt ? entry_at<BN>(x, h, P) : 0u;
 #pragma unroll 1
       for (int k = 0; k < ns; ++k) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[X], sn & 1, abort_flag, P.status))) { ok = false; break; }
-        ++sn;
-        tc_fence_after();
         uint32_t e[BPS];
         bool mem[BPS];
         bool any_mem = false;
+        bool slot_mem = false;   // one of this slot's query blocks selected an entry of the step
 #pragma unroll
         for (int h = 0; h < BPS; ++h) {
           e[h] = e_next[h];
@@ -474,7 +524,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (k + 1 < ns) e_next[h] = idx < x.cnt ? entry_at<BN>(x, idx, P) : 0u;
           mem[h] = (e[h] >> (16 + qb)) & 1u;     // warp-uniform: a warp's rows share qb
           any_mem |= mem[h];
+          slot_mem |= ((e[h] >> 16) & kSlotMask) != 0u;
         }
+        // With 64-token blocks the MMA warp computes neither S nor P.V for a step none
+        // of the slot's query blocks selected (the same test on the same entries), so
+        // there is nothing to wait for. slot_mem is warp-uniform (the entries are).
+        if (BN == 64 && !slot_mem) continue;
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[X], sn & 1, abort_flag, P.status))) { ok = false; break; }
+        ++sn;
+        tc_fence_after();
         // any_mem is warp-uniform: it depends only on the step's union entries
         // (the same for every lane) and on qb, which all 32 rows of a warp share
         // (32 divides BN). The S loads and P stores below therefore run on full warps.
@@ -681,6 +739,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+        }
+        if (!(l_run > 0.f)) {   // a row no processed step reached: O was never written
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] = 0u;
         }
         if (store) {
 #pragma unroll
