@@ -51,12 +51,12 @@ METRIC = "sparse attn ms/call & effective TFLOP/s (Wan-14B 720p shape) vs own de
 # head's K and V) fits in L2 at both sizes, so the re-read factor carries over.
 # After any change of the source the traffic is unknown and reported as null.
 ATTN_TRAFFIC = {
-    # 1,022,956,288 read + 319,735,296 written; Q, K, V, O at 2 B x 40 x 256 x 128 x 128
-    "bf16": {"bytes_480p": 1022956288 + 319735296, "algorithmic_480p": 4 * 40 * 256 * 128 * 128 * 2,
-             "src": "92c0efc2d48a10bf"},
-    # 846,715,136 read + 315,955,968 written; Q, K, O at 2 B and the E4M3 V at 1 B
-    "fp8v": {"bytes_480p": 846715136 + 315955968, "algorithmic_480p": 7 * 40 * 256 * 128 * 128,
-             "src": "92c0efc2d48a10bf"},
+    # 1,022,893,568 read + 320,081,408 written; Q, K, V, O at 2 B x 40 x 256 x 128 x 128
+    "bf16": {"bytes_480p": 1022893568 + 320081408, "algorithmic_480p": 4 * 40 * 256 * 128 * 128 * 2,
+             "src": "fa3c8bbf00b238b1"},
+    # 846,904,576 read + 315,604,736 written; Q, K, O at 2 B and the E4M3 V at 1 B
+    "fp8v": {"bytes_480p": 846904576 + 315604736, "algorithmic_480p": 7 * 40 * 256 * 128 * 128,
+             "src": "fa3c8bbf00b238b1"},
 }
 ATTN_SRC = os.path.join(ROOT, "block_sparse_attention_video_b200", "csrc", "attn_sm100.cu")
 
