@@ -56,7 +56,9 @@ def test_invalid_lists_are_reported_and_valid_rows_kept(w):
     # the broken rows' neighbours in other query blocks are untouched by the clamping
     mask = mask_from_lists(good_idx.cpu().numpy(), good_cnt.cpu().numpy(), nb)
     to_np = lambda t: t.float().cpu().numpy()
-    ref = O.masked_attention(to_np(qp), to_np(kp), to_np(vp), mask, w.N, w.block, 1.0 / math.sqrt(w.d))
+    perm = O.tile_order(*w.grid, *w.tile)      # the oracle's own permutation of the seeded inputs
+    ref = O.masked_attention(*(O.permute(to_np(x), perm, w.block) for x in (q, k, v)), mask, w.N, w.block,
+                             1.0 / math.sqrt(w.d))
     bs = w.block
     for (b, h, i) in [(0, 0, 0), (0, 1, 0), (0, 0, nb - 1)]:
         rows = slice(i * bs, min((i + 1) * bs, w.N))

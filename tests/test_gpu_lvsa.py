@@ -80,10 +80,14 @@ def test_sparse_attention_over_lvsa_lists():
     ws = F.alloc_workspace(F.fvattn_workspace_bytes(F.FVATTN_OP_SPARSE_FWD, w.B, w.H, w.N, w.d, w.block), "cuda")
     F.fvattn_sparse_fwd(qp, kp, vp, op, kv_idx, kv_cnt, w.N, w.block, ws)
     assert F.fvattn_workspace_status(ws) == F.FVATTN_OK
+    perm = O.tile_order(*w.grid, *w.tile)
+    want = L.lvsa_block_mask(perm, w.grid, w.block, 0, 8, 1)       # the oracle's mask
     mask = mask_from_lists(kv_idx.cpu().numpy(), kv_cnt.cpu().numpy(), grid.nb)
-    assert 0.2 < mask.mean() < 0.9
+    assert all(np.array_equal(mask[0, h], want) for h in range(w.H))
+    assert 0.2 < want.mean() < 0.9
     to_np = lambda t: t.float().cpu().numpy()
-    ref = O.masked_attention(to_np(qp), to_np(kp), to_np(vp), mask, w.N, w.block, 1.0 / math.sqrt(w.d))
+    ref = O.masked_attention(*(O.permute(to_np(x), perm, w.block) for x in (q, k, v)),
+                             np.broadcast_to(want, mask.shape), w.N, w.block, 1.0 / math.sqrt(w.d))
     mx, mean = attention_errors(to_np(op)[:, :, :w.N], ref[:, :, :w.N])
     assert mx <= BF16_MAX_ABS and mean <= BF16_MEAN_ABS, (mx, mean)
     print(f"lvsa attention: density {mask.mean():.3f} max_abs {mx:.2e} mean_abs {mean:.2e}")
