@@ -17,6 +17,7 @@ import numpy as np
 
 from oracle.mask_parity import BORDER_CUM, BORDER_REL, borderline_ceiling, mask_from_lists  # noqa: F401
 from oracle.mask_parity import compare_masks as _compare
+from oracle.fvattn_oracle import permute as _permute, tile_order as _tile_order
 
 BF16_MAX_ABS = 2e-2
 BF16_MEAN_ABS = 2e-3
@@ -58,3 +59,10 @@ def assert_mask_parity(res: dict, label: str) -> str:
 def attention_errors(gpu: np.ndarray, ref: np.ndarray):
     err = np.abs(gpu.astype(np.float64) - ref)
     return float(err.max()), float(err.mean())
+
+
+def oracle_permuted(w, *tensors):
+    """The seeded inputs in the oracle's own 3-D tile order, padded to nb*bs: the oracle's
+    inputs never come from the library's permutation."""
+    perm = _tile_order(*w.grid, *w.tile)
+    return tuple(_permute(t.detach().float().cpu().numpy(), perm, w.block) for t in tensors)

@@ -25,7 +25,7 @@ import torch
 
 import oracle as O
 import synthetic as S
-from parity import mask_from_lists
+from parity import mask_from_lists, oracle_permuted
 from test_gpu_parity import BS64, ODD, ODD128, PEAKY, _np, _route_gpu
 
 pytestmark = pytest.mark.gpu
@@ -102,7 +102,7 @@ def test_sparse_block_lse_and_importance_match_oracle(w):
     F.fvattn_permute(v, vp, grid)
     blse, _, imp = _diag_gpu(w, qp, kp, vp, kv_idx, kv_cnt)
     mask = mask_from_lists(kv_idx.cpu().numpy(), kv_cnt.cpu().numpy(), grid.nb)
-    qn, kn = _np(qp), _np(kp)
+    qn, kn = oracle_permuted(w, q, k)   # the oracle's own tile order of the seeded inputs
     rows = [(b, h, i) for b in range(w.B) for h in range(w.H) for i in range(grid.nb)]
     wb, wi = _check_rows(w, qn, kn, mask, blse, imp, rows)
     print(f"{w.name}: density {mask.mean():.3f} max |d block_lse| {wb:.2e} max |d importance| {wi:.2e}")
@@ -117,7 +117,7 @@ def test_dense_importance_and_recall_of_routed_mask(w):
     nb = grid.nb
     blse, _, imp = _diag_gpu(w, qp, kp, vp)
     full = np.ones((w.B, w.H, nb, nb), bool)
-    qn, kn = _np(qp), _np(kp)
+    qn, kn = oracle_permuted(w, q, k)   # the oracle's own tile order of the seeded inputs
     rows = [(b, h, i) for b in range(w.B) for h in range(w.H) for i in range(nb)]
     _check_rows(w, qn, kn, full, blse, imp, rows)
     rec = _recall_gpu(w, imp, kv_idx, kv_cnt)
@@ -145,7 +145,7 @@ def test_importance_and_recall_sampled_480p():
     rng = np.random.default_rng(5)
     rows = [(0, int(h), int(i)) for h, i in zip(rng.integers(0, w.H, 12), rng.integers(0, nb, 12))]
     rows.append((0, w.H - 1, nb - 1))               # the ragged last block
-    qn, kn = _np(qp), _np(kp)
+    qn, kn = oracle_permuted(w, q, k)   # the oracle's own tile order of the seeded inputs
     _check_rows(w, qn, kn, mask, blse, imp, rows)
     imp_gpu = torch.from_numpy(imp)
     sums = imp_gpu.sum(-1)

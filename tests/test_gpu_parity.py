@@ -17,7 +17,7 @@ import torch
 import oracle as O
 import synthetic as S
 from parity import (BF16_MAX_ABS, BF16_MEAN_ABS, FP32_MAX_ABS, assert_mask_parity, attention_errors,
-                    check_lists_valid, compare_masks, mask_from_lists)
+                    check_lists_valid, compare_masks, mask_from_lists, oracle_permuted)
 
 pytestmark = pytest.mark.gpu
 
@@ -136,8 +136,9 @@ def test_route_uniform_scores_tie_break():
 
 
 # ----------------------------------------------------------------- attention
-def _check_attention(w, qp, kp, vp, op, mask, blocks, tol_max, tol_mean):
-    qpn, kpn, vpn = _np(qp), _np(kp), _np(vp)
+def _check_attention(w, q, k, v, op, mask, blocks, tol_max, tol_mean):
+    # oracle inputs: the seeded q, k, v in the oracle's own tile order
+    qpn, kpn, vpn = oracle_permuted(w, q, k, v)
     ref = O.masked_attention(qpn, kpn, vpn, mask, w.N, w.block, 1.0 / math.sqrt(w.d), blocks=blocks)
     got = _np(op)
     rows = np.zeros(ref.shape[:-1], dtype=bool)
@@ -176,9 +177,9 @@ def test_sparse_and_dense_attention_all_blocks(w):
     tol = (FP32_MAX_ABS, FP32_MAX_ABS) if w.dtype == "fp32" else (BF16_MAX_ABS, BF16_MEAN_ABS)
     op, _ = _attn_gpu(w, qp, kp, vp, kv_idx, kv_cnt)
     mask = mask_from_lists(kv_idx.cpu().numpy(), kv_cnt.cpu().numpy(), nb)
-    _check_attention(w, qp, kp, vp, op, mask, blocks, *tol)
+    _check_attention(w, q, k, v, op, mask, blocks, *tol)
     opd, _ = _attn_gpu(w, qp, kp, vp)
-    _check_attention(w, qp, kp, vp, opd, np.ones_like(mask), blocks, *tol)
+    _check_attention(w, q, k, v, opd, np.ones_like(mask), blocks, *tol)
 
 
 @pytest.mark.parametrize("name", ["wan1.3b-480p", "wan14b-480p"])
@@ -193,16 +194,17 @@ def test_tensor_core_attention_sampled(name):
     mask = mask_from_lists(kv_idx.cpu().numpy(), cnt, nb)
     blocks = _sample_blocks(w, nb, cnt, per_head=3)
     op, lse = _attn_gpu(w, qp, kp, vp, kv_idx, kv_cnt, lse=True)
-    _check_attention(w, qp, kp, vp, op, mask, blocks, BF16_MAX_ABS, BF16_MEAN_ABS)
+    _check_attention(w, q, k, v, op, mask, blocks, BF16_MAX_ABS, BF16_MEAN_ABS)
     # lse of one row against the oracle's logits
     b, h, i = blocks[0]
     r = i * w.block
     cols = np.concatenate([np.arange(j * w.block, min((j + 1) * w.block, w.N)) for j in np.nonzero(mask[b, h, i])[0]])
-    logits = (_np(qp)[b, h, r].astype(np.float64) @ _np(kp)[b, h, cols].astype(np.float64).T) / math.sqrt(w.d)
+    qo, ko = oracle_permuted(w, q, k)
+    logits = (qo[b, h, r].astype(np.float64) @ ko[b, h, cols].astype(np.float64).T) / math.sqrt(w.d)
     ref_lse = logits.max() + math.log(np.exp(logits - logits.max()).sum())
     assert abs(float(lse[b, h, r]) - ref_lse) < 1e-3
     opd, _ = _attn_gpu(w, qp, kp, vp)
-    _check_attention(w, qp, kp, vp, opd, np.ones_like(mask), blocks[: 4 * w.H: 4],
+    _check_attention(w, q, k, v, opd, np.ones_like(mask), blocks[: 4 * w.H: 4],
                      BF16_MAX_ABS, BF16_MEAN_ABS)
 
 
@@ -289,7 +291,7 @@ def test_batch_of_two_tensor_core():
     cnt = kv_cnt.cpu().numpy()
     mask = mask_from_lists(kv_idx.cpu().numpy(), cnt, nb)
     op, _ = _attn_gpu(w, qp, kp, vp, kv_idx, kv_cnt)
-    _check_attention(w, qp, kp, vp, op, mask, _sample_blocks(w, nb, cnt, per_head=4),
+    _check_attention(w, q, k, v, op, mask, _sample_blocks(w, nb, cnt, per_head=4),
                      BF16_MAX_ABS, BF16_MEAN_ABS)
 
 
