@@ -45,18 +45,19 @@ METRIC = "sparse attn ms/call & effective TFLOP/s (Wan-14B 720p shape) vs own de
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
 # launch from a one-pass ncu capture on the Wan-14B 480p shape (the size a
 # capture may hold), with the algorithmic bytes of that launch (Q, K, V read
-# once, O written once) and the sha256 prefix of the kernel source it was taken
-# on. A 720p launch's traffic is reported as the 480p traffic scaled by the ratio
-# of algorithmic bytes: the working set of the work units in flight (about one
-# head's K and V) fits in L2 at both sizes, so the re-read factor carries over.
-# After any change of the source the traffic is unknown and reported as null.
+# once, O written once) and the prefix of _code_hash of the kernel source it was
+# taken on (comments do not count). A 720p launch's traffic is reported as the
+# 480p traffic scaled by the ratio of algorithmic bytes: the working set of the
+# work units in flight (about one head's K and V) fits in L2 at both sizes, so the
+# re-read factor carries over. After any change of the code the traffic is unknown
+# and reported as null.
 ATTN_TRAFFIC = {
     # 1,022,893,568 read + 320,081,408 written; Q, K, V, O at 2 B x 40 x 256 x 128 x 128
     "bf16": {"bytes_480p": 1022893568 + 320081408, "algorithmic_480p": 4 * 40 * 256 * 128 * 128 * 2,
-             "src": "fa3c8bbf00b238b1"},
+             "src": "729c0bf9fa452b22"},
     # 846,904,576 read + 315,604,736 written; Q, K, O at 2 B and the E4M3 V at 1 B
     "fp8v": {"bytes_480p": 846904576 + 315604736, "algorithmic_480p": 7 * 40 * 256 * 128 * 128,
-             "src": "fa3c8bbf00b238b1"},
+             "src": "729c0bf9fa452b22"},
 }
 ATTN_SRC = os.path.join(ROOT, "block_sparse_attention_video_b200", "csrc", "attn_sm100.cu")
 
@@ -74,6 +75,17 @@ def _frac_at_clock(achieved_tflops: float, clocks, dev):
     return achieved_tflops / peak
 
 
+def _code_hash(text: str) -> str:
+    """sha256 of a C++/CUDA source with its comments and blank lines removed, so that an
+    edit of comments alone keeps a recorded measurement of the code valid."""
+    import hashlib
+    import re
+    t = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    t = re.sub(r"//[^\n]*", "", t)
+    lines = [ln.rstrip() for ln in t.splitlines() if ln.strip()]
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()
+
+
 def _attn_traffic(kind: str, algorithmic_bytes: float):
     """(scaled DRAM bytes per launch, note) for the current kernel source, or (None, why)."""
     import hashlib
@@ -81,12 +93,12 @@ def _attn_traffic(kind: str, algorithmic_bytes: float):
     if rec is None or rec["bytes_480p"] is None:
         return None, "no capture recorded"
     try:
-        with open(ATTN_SRC, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
+        with open(ATTN_SRC) as f:
+            sha = _code_hash(f.read())
     except OSError:
         return None, "kernel source not found"
     if not sha.startswith(rec["src"]):
-        return None, "kernel source changed since the capture"
+        return None, "kernel code changed since the capture"
     ratio = rec["bytes_480p"] / rec["algorithmic_480p"]
     return ratio * algorithmic_bytes, (f"ncu one-pass DRAM bytes at the Wan-14B 480p shape "
                                        f"({rec['bytes_480p'] / 1e9:.3f} GB, {ratio:.3f}x its algorithmic bytes), "

@@ -1,6 +1,6 @@
 // attn_sm100.cu -- block-sparse attention forward on the Blackwell tensor cores
-// (tcgen05 MMA with TMEM accumulators, TMA-fed), bf16 inputs, d = 128, blocks of
-// BN = 64 or 128 tokens [FVAttn §2.1: only selected (query block, key block)
+// (tcgen05 MMA with TMEM accumulators, TMA-fed), bf16 inputs, head dimension
+// d = 64 or 128, blocks of BN = 64 or 128 tokens [FVAttn §2.1: only selected (query block, key block)
 // pairs are evaluated; GSRS §3.2: unselected blocks are skipped in the tiling
 // loop; GSRS §A.1: online softmax, rescaling earlier partial results when the
 // max grows].
@@ -30,7 +30,9 @@
 //
 // MMA order per unit: S0(0) S1(0), then for k >= 1: PV0(k-1) S0(k) PV1(k-1)
 // S1(k), and finally PV0(last) PV1(last): the exponentials of one slot overlap
-// the other slot's MMAs.
+// the other slot's MMAs. With BN = 64 a slot leaves out its S and P.V of a step
+// that neither of its two query blocks selected (the softmax warps skip that
+// step too); Q and O of both slots are released after the unit's last MMA.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512).
 // P (bf16, two per 32-bit column) overwrites the first 64 columns of S and is
 // the A operand of the P.V MMA straight from TMEM.

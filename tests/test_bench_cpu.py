@@ -3,7 +3,6 @@ sweep's configurations, the traffic record keyed by the attention source's hash,
 and the reference arm's JSON line on a bounded sample."""
 
 import argparse
-import hashlib
 import json
 
 import pytest
@@ -38,8 +37,8 @@ def test_sweep_covers_p_kmin_and_block_sizes():
 
 
 def test_traffic_is_reported_only_for_the_captured_source():
-    with open(bench.ATTN_SRC, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()
+    with open(bench.ATTN_SRC) as f:
+        sha = bench._code_hash(f.read())
     for kind, rec in bench.ATTN_TRAFFIC.items():
         got, note = bench._attn_traffic(kind, 2.0e9)
         if rec["bytes_480p"] is not None and sha.startswith(rec["src"]):
@@ -112,3 +111,9 @@ def test_oracle_check_on_the_oracles_own_result():
     rng = np.random.default_rng(0)
     _, err2, *_ = bench.oracle_check(w, q, k, v, idx, cnt, op, [0], per_head=nb, rng=rng)
     assert err2["max_abs"] >= 0.999 and not err2["within_tolerance"]
+
+
+def test_code_hash_ignores_comments_only():
+    code = "int f(int x) {\n  return x + 1;  // add one\n}\n"
+    assert bench._code_hash(code) == bench._code_hash("/* doc */\nint f(int x) {\n  return x + 1;\n}\n")
+    assert bench._code_hash(code) != bench._code_hash(code.replace("+ 1", "+ 2"))
